@@ -1,0 +1,253 @@
+// C-ABI entry points declared in include/jattn.h: argument validation (all of
+// it before any launch), TMA tensor-map encoding, launches on the caller's
+// stream, and the per-device status word.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "jattn.h"
+#include "jattn_internal.h"
+
+namespace {
+
+// Device errors found by the kernels (JATTN_DEV_* bits).  One word per
+// device: every module load gets its own copy.
+__device__ uint32_t g_status_word;
+
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;   // 2 s per pipeline wait
+constexpr int kMaxDevices = 64;
+
+uint32_t* status_ptr() {
+  static uint32_t* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<uint32_t*>(p);
+  }
+  return ptrs[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+jattn_status check_shape(const jattn_shape* s) {
+  if (s == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (s->B < 1 || s->H < 1 || s->S_txt < 0 || s->S_img < 0 || s->S_ref < 0) return JATTN_ERR_INVALID_ARG;
+  const int64_t S = static_cast<int64_t>(s->S_txt) + s->S_img + s->S_ref;
+  if (S < 1 || S > (1 << 24)) return JATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(s->B) * s->H > 65535) return JATTN_ERR_INVALID_ARG;   // grid.y
+  if (s->d != 64 && s->d != 128) return JATTN_ERR_UNSUPPORTED;
+  return JATTN_OK;
+}
+
+int total_S(const jattn_shape* s) { return s->S_txt + s->S_img + s->S_ref; }
+int n_blocks(int S) { return (S + JATTN_BLOCK - 1) / JATTN_BLOCK; }
+
+// [BH][S][d] tensor map with (d-inner) boxes of box_inner elements x 128 rows.
+jattn_status make_map(CUtensorMap* m, const void* base, int BH, int S, int d, int elem_bytes) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return JATTN_ERR_CUDA;
+  const int row_bytes = d * elem_bytes;
+  const int sw_bytes = row_bytes >= 128 ? 128 : 64;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * S};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(sw_bytes / elem_bytes), 128u, 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUtensorMapSwizzle sw = sw_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? JATTN_OK : JATTN_ERR_CUDA;
+}
+
+float resolve_scale(float softmax_scale, int d) {
+  return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
+}
+
+}  // namespace
+
+extern "C" {
+
+jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                            const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
+                            jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream) {
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  if (split == nullptr || pos == nullptr || q == nullptr || k == nullptr || v == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!(theta > 0.f) || !std::isfinite(theta)) return JATTN_ERR_INVALID_ARG;
+  if (split[0] < 0 || split[1] < 0 || split[2] < 0 || (split[0] | split[1] | split[2]) & 1 ||
+      split[0] + split[1] + split[2] != shape->d)
+    return JATTN_ERR_INVALID_ARG;
+  const void* parts[3] = {qkv_txt, qkv_img, qkv_ref};
+  const int lens[3] = {shape->S_txt, shape->S_img, shape->S_ref};
+  for (int i = 0; i < 3; ++i) {
+    if (lens[i] > 0 && parts[i] == nullptr) return JATTN_ERR_INVALID_ARG;
+    if (lens[i] > 0 && !aligned16(parts[i])) return JATTN_ERR_ALIGNMENT;
+  }
+  if (out_dtype != JATTN_BF16 && out_dtype != JATTN_FP16 && out_dtype != JATTN_E4M3) return JATTN_ERR_UNSUPPORTED;
+  if (out_dtype == JATTN_E4M3 && scales == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(pos)) return JATTN_ERR_ALIGNMENT;
+
+  jattn::RopeParams p{};
+  for (int i = 0; i < 3; ++i) {
+    p.src[i] = static_cast<const __nv_bfloat16*>(parts[i]);
+    p.S_part[i] = lens[i];
+    p.split[i] = split[i];
+  }
+  p.B = shape->B;
+  p.H = shape->H;
+  p.S = total_S(shape);
+  p.d = shape->d;
+  p.nblk = n_blocks(p.S);
+  p.pos = pos;
+  p.theta = static_cast<double>(theta);
+  p.dst[0] = q;
+  p.dst[1] = k;
+  p.dst[2] = v;
+  p.scales = scales;
+  p.status = status_ptr();
+  if (p.status == nullptr) return JATTN_ERR_CUDA;
+  const int kind = out_dtype == JATTN_FP16 ? 0 : (out_dtype == JATTN_BF16 ? 1 : 2);
+  return jattn::launch_rope_qkv(p, kind, static_cast<cudaStream_t>(stream)) == cudaSuccess ? JATTN_OK
+                                                                                          : JATTN_ERR_CUDA;
+}
+
+jattn_status jattn_quant_fp8(const jattn_shape* shape, jattn_dtype in_dtype, const void* x, void* x8,
+                             float* scales, void* stream) {
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  if (x == nullptr || x8 == nullptr || scales == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (in_dtype != JATTN_BF16 && in_dtype != JATTN_FP16) return JATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x8)) return JATTN_ERR_ALIGNMENT;
+  jattn::QuantParams p{};
+  p.x = x;
+  p.x8 = x8;
+  p.scales = scales;
+  p.BH = shape->B * shape->H;
+  p.S = total_S(shape);
+  p.d = shape->d;
+  p.nblk = n_blocks(p.S);
+  return jattn::launch_quant_fp8(p, in_dtype == JATTN_BF16, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? JATTN_OK
+             : JATTN_ERR_CUDA;
+}
+
+static jattn_status fwd_common(const jattn_shape* shape, const void* q, const void* k, const void* v, void* o,
+                               float* lse, float softmax_scale, jattn::FwdParams& p) {
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return JATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(softmax_scale)) return JATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return JATTN_ERR_ALIGNMENT;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return JATTN_ERR_ALIGNMENT;
+  p.B = shape->B;
+  p.H = shape->H;
+  p.S = total_S(shape);
+  p.n_tiles = n_blocks(p.S);
+  p.scale_log2 = resolve_scale(softmax_scale, shape->d) * 1.4426950408889634f;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.status = status_ptr();
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (p.status == nullptr) return JATTN_ERR_CUDA;
+  return JATTN_OK;
+}
+
+jattn_status jattn_fwd_bf16(const jattn_shape* shape, jattn_dtype in_dtype, const void* q, const void* k,
+                            const void* v, void* o, float* lse, float softmax_scale, void* stream) {
+  if (in_dtype != JATTN_BF16 && in_dtype != JATTN_FP16) return JATTN_ERR_UNSUPPORTED;
+  jattn::FwdParams p{};
+  jattn_status st = fwd_common(shape, q, k, v, o, lse, softmax_scale, p);
+  if (st != JATTN_OK) return st;
+  CUtensorMap tq, tk, tv;
+  const int BH = p.B * p.H;
+  if ((st = make_map(&tq, q, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
+  return jattn::launch_fwd_f16(p, shape->d, in_dtype == JATTN_BF16, tq, tk, tv,
+                               static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? JATTN_OK
+             : JATTN_ERR_CUDA;
+}
+
+jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void* k8, const void* v8,
+                           const float* scales, void* o, float* lse, float softmax_scale, void* stream) {
+  if (scales == nullptr || (reinterpret_cast<uintptr_t>(scales) & 3u)) return JATTN_ERR_INVALID_ARG;
+  jattn::FwdParams p{};
+  jattn_status st = fwd_common(shape, q8, k8, v8, o, lse, softmax_scale, p);
+  if (st != JATTN_OK) return st;
+  p.scales = scales;
+  CUtensorMap tq, tk, tv;
+  const int BH = p.B * p.H;
+  if ((st = make_map(&tq, q8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
+  return jattn::launch_fwd_fp8(p, shape->d, tq, tk, tv, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? JATTN_OK
+             : JATTN_ERR_CUDA;
+}
+
+jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits) {
+  uint32_t* ptr = status_ptr();
+  if (ptr == nullptr) return JATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return JATTN_ERR_CUDA;
+  uint32_t w = 0;
+  if (cudaMemcpy(&w, ptr, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return JATTN_ERR_CUDA;
+  if (clear && cudaMemset(ptr, 0, sizeof(uint32_t)) != cudaSuccess) return JATTN_ERR_CUDA;
+  if (bits != nullptr) *bits = w;
+  if (w & JATTN_DEV_TIMEOUT) return JATTN_ERR_TIMEOUT;
+  if (w & JATTN_DEV_RANGE) return JATTN_ERR_RANGE;
+  return JATTN_OK;
+}
+
+jattn_status jattn_selftest_wait_timeout(int32_t limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 10000) return JATTN_ERR_INVALID_ARG;
+  uint32_t* ptr = status_ptr();
+  if (ptr == nullptr) return JATTN_ERR_CUDA;
+  return jattn::launch_selftest_wait(ptr, static_cast<uint64_t>(limit_ms) * 1000000ull,
+                                     static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? JATTN_OK
+             : JATTN_ERR_CUDA;
+}
+
+const char* jattn_status_string(jattn_status s) {
+  switch (s) {
+    case JATTN_OK: return "ok";
+    case JATTN_ERR_INVALID_ARG: return "invalid argument";
+    case JATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case JATTN_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case JATTN_ERR_CUDA: return "CUDA error";
+    case JATTN_ERR_TIMEOUT: return "device wait timed out";
+    case JATTN_ERR_RANGE: return "value out of 16-bit range (saturated)";
+  }
+  return "unknown status";
+}
+
+const char* jattn_version(void) { return "0.1.0"; }
+
+}  // extern "C"

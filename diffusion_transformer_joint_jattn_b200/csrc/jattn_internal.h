@@ -1,0 +1,54 @@
+// Parameter blocks and launchers shared by the C-ABI layer (jattn_api.cu)
+// and the kernel translation units.  Not part of the public interface.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+namespace jattn {
+
+struct RopeParams {
+  const __nv_bfloat16* src[3];  // txt, img, ref streams [B, S_part, 3, H, d]
+  int S_part[3];
+  int B, H, S, d, nblk;
+  const int32_t* pos;           // [S, 3]
+  double theta;
+  int split[3];
+  void* dst[3];                 // q, k, v [B, H, S, d]
+  float* scales;                // e4m3 output: [3][B][H][nblk]
+  uint32_t* status;
+};
+
+struct QuantParams {
+  const void* x;                // [BH, S, d] 16-bit
+  void* x8;                     // [BH, S, d] e4m3
+  float* scales;                // [BH][nblk]
+  int BH, S, d, nblk;
+};
+
+struct FwdParams {
+  int B, H, S, n_tiles;         // n_tiles = ceil(S / 128)
+  float scale_log2;             // softmax_scale * log2(e)
+  __nv_bfloat16* o;             // [B, S, H, d]
+  float* lse;                   // [B, H, S] or null
+  const float* scales;          // fp8: [3][B][H][n_tiles]
+  uint32_t* status;
+  uint64_t timeout_ns;
+};
+
+// out_kind: 0 = fp16, 1 = bf16, 2 = e4m3
+cudaError_t launch_rope_qkv(const RopeParams& p, int out_kind, cudaStream_t st);
+cudaError_t launch_quant_fp8(const QuantParams& p, bool in_bf16, cudaStream_t st);
+
+// 16-bit forward (in_bf16 selects the operand type) and e4m3 forward.  The
+// tensor maps describe q, k, v as 3-D [BH][S][d] with 128-row boxes.
+cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtensorMap& tq,
+                           const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st);
+cudaError_t launch_fwd_fp8(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                           const CUtensorMap& tv, cudaStream_t st);
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
+
+}  // namespace jattn

@@ -1,0 +1,318 @@
+// Prologue kernels: joint-sequence assembly + 2D axial RoPE on Q/K, with the
+// output either in a 16-bit type or quantised to e4m3 with one fp32 scale
+// per (batch, head, 128-token block); and the standalone block quantiser.
+//
+// Method ("Speed Up Image Generation with FLUX 3 Image Klein on NVIDIA
+// Blackwell GPUs"): the text, target-image and reference-image streams are
+// joined for joint attention (section "FLUX 3 inference with TensorRT LLM
+// VisualGen"); rotary embeddings act on the query and key projections
+// (section "GEMM kernel optimization"); FP8 Q/K/V feed the quantised
+// attention (section "Quantized and sparse attention").
+//
+// Design: HBM-bound streaming.  One CTA owns one 128-token block of one batch
+// entry and walks all 3*H (Q/K/V, head) tiles of it, so each (token, pair)
+// cos/sin is computed once per CTA and lives in registers; loads and stores
+// are 16-byte vectors, coalesced along d; the next tile's loads are issued
+// before the current tile is processed.  For e4m3 output the tile's amax is
+// reduced across the CTA before its codes are written, so every input byte is
+// read exactly once.
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_fp16.h>
+#include <cuda_bf16.h>
+
+#include "jattn.h"
+#include "jattn_internal.h"
+
+namespace jattn {
+
+namespace {
+
+constexpr int kTok = JATTN_BLOCK;   // tokens per CTA (= FP8 scale block)
+constexpr int kTokPerThread = 4;
+
+enum OutKind { kOutF16 = 0, kOutBF16 = 1, kOutE4M3 = 2 };
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    x[2 * i] = __uint_as_float(w[i] << 16);
+    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+// Two fp32 -> two e4m3 (RNE, saturating to +-448); `a` lands in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Axis, index inside the axis span and span width of channel pair `pair`
+// (0 .. d/2-1); spans are laid out t, row, col.
+__device__ __forceinline__ void pair_axis(int pair, int n0, int n1, int n2, int& axis, int& i, int& n) {
+  if (pair < n0 / 2) { axis = 0; i = pair; n = n0; }
+  else if (pair < (n0 + n1) / 2) { axis = 1; i = pair - n0 / 2; n = n1; }
+  else { axis = 2; i = pair - (n0 + n1) / 2; n = n2; }
+}
+
+// cos/sin of pos_axis * theta^(-2i/n): the angle is formed and reduced to
+// [-pi, pi] in fp64, then rotated with the fp32 sincos.
+__device__ __forceinline__ void pair_cos_sin(int32_t pos_axis, int i, int n, double theta,
+                                             float& c, float& s) {
+  const double omega = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(n));
+  const double ang = static_cast<double>(pos_axis) * omega;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double r = ang - rint(ang / two_pi) * two_pi;
+  sincosf(static_cast<float>(r), &s, &c);
+}
+
+// OUT: output kind.  D: head dimension.
+template <int D, int OUT>
+__global__ void __launch_bounds__(D / 8 * kTok / kTokPerThread)
+rope_qkv_kernel(const RopeParams p) {
+  constexpr int CG = D / 8;                           // 16-byte chunks per row
+  constexpr int NT = CG * kTok / kTokPerThread;       // threads
+  constexpr int ROWS_PER_PASS = kTok / kTokPerThread; // tokens covered by one pass
+  constexpr int NWARP = NT / 32;
+  __shared__ float red[2][NWARP];
+
+  const int tid = threadIdx.x;
+  const int cg = tid % CG;
+  const int trow = tid / CG;
+  const int blk = blockIdx.x;
+  const int b = blockIdx.y;
+  const int H = p.H, S = p.S;
+  const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
+
+  // Per-token source row base (element offset of [b, local, 0, 0, 0] in its
+  // stream) and validity.
+  const __nv_bfloat16* src[kTokPerThread];
+  int tok[kTokPerThread];
+  bool valid[kTokPerThread];
+  float cs[kTokPerThread][4], sn[kTokPerThread][4];
+#pragma unroll
+  for (int i = 0; i < kTokPerThread; ++i) {
+    const int t = blk * kTok + trow + i * ROWS_PER_PASS;
+    tok[i] = t;
+    valid[i] = t < S;
+    const __nv_bfloat16* base = p.src[0];
+    int len = p.S_part[0], local = t;
+    if (t >= p.S_part[0]) { base = p.src[1]; len = p.S_part[1]; local = t - p.S_part[0]; }
+    if (t >= p.S_part[0] + p.S_part[1]) { base = p.src[2]; len = p.S_part[2]; local = t - p.S_part[0] - p.S_part[1]; }
+    src[i] = valid[i] ? base + (static_cast<size_t>(b) * len + local) * 3 * H * D + cg * 8 : nullptr;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cs[i][j] = 1.f;
+      sn[i][j] = 0.f;
+      if (valid[i]) {
+        int axis, ii, n;
+        pair_axis(cg * 4 + j, n0, n1, n2, axis, ii, n);
+        pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs[i][j], sn[i][j]);
+      }
+    }
+  }
+
+  const int items = 3 * H;
+  uint4 nxt[kTokPerThread];
+  auto load_item = [&](int item, uint4 (&buf)[kTokPerThread]) {
+    const int which = item / H, h = item % H;
+    const size_t off = static_cast<size_t>(which * H + h) * D;
+#pragma unroll
+    for (int i = 0; i < kTokPerThread; ++i)
+      buf[i] = valid[i] ? __ldg(reinterpret_cast<const uint4*>(src[i] + off)) : make_uint4(0, 0, 0, 0);
+  };
+  load_item(0, nxt);
+  bool range_hit = false;
+
+  for (int item = 0; item < items; ++item) {
+    uint4 cur[kTokPerThread];
+#pragma unroll
+    for (int i = 0; i < kTokPerThread; ++i) cur[i] = nxt[i];
+    if (item + 1 < items) load_item(item + 1, nxt);
+    const int which = item / H, h = item % H;
+
+    float x[kTokPerThread][8];
+#pragma unroll
+    for (int i = 0; i < kTokPerThread; ++i) {
+      bf16x8_to_f32(cur[i], x[i]);
+      if (which < 2) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float a = x[i][2 * j], bb = x[i][2 * j + 1];
+          x[i][2 * j] = a * cs[i][j] - bb * sn[i][j];
+          x[i][2 * j + 1] = a * sn[i][j] + bb * cs[i][j];
+        }
+      }
+    }
+    const size_t row0 = (static_cast<size_t>(b) * H + h) * S;
+
+    if constexpr (OUT == kOutE4M3) {
+      float am = 0.f;
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[i][e]));
+      am = warp_max(am);
+      float* slot = red[item & 1];
+      if ((tid & 31) == 0) slot[tid >> 5] = am;
+      __syncthreads();
+      am = 0.f;
+#pragma unroll
+      for (int w = 0; w < NWARP; ++w) am = fmaxf(am, slot[w]);
+      const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      const float inv = am > 0.f ? __fdiv_rn(448.0f, am) : 1.0f;
+      uint8_t* dst = static_cast<uint8_t*>(which == 0 ? p.dst[0] : (which == 1 ? p.dst[1] : p.dst[2]));
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i) {
+        if (!valid[i]) continue;
+        uint2 o;
+        o.x = pack_e4m3x2(__fmul_rn(x[i][0], inv), __fmul_rn(x[i][1], inv)) |
+              (pack_e4m3x2(__fmul_rn(x[i][2], inv), __fmul_rn(x[i][3], inv)) << 16);
+        o.y = pack_e4m3x2(__fmul_rn(x[i][4], inv), __fmul_rn(x[i][5], inv)) |
+              (pack_e4m3x2(__fmul_rn(x[i][6], inv), __fmul_rn(x[i][7], inv)) << 16);
+        *reinterpret_cast<uint2*>(dst + (row0 + tok[i]) * D + cg * 8) = o;
+      }
+      if (tid == 0)
+        p.scales[((static_cast<size_t>(which) * p.B + b) * H + h) * p.nblk + blk] = scale;
+    } else {
+      uint16_t* dst = static_cast<uint16_t*>(which == 0 ? p.dst[0] : (which == 1 ? p.dst[1] : p.dst[2]));
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i) {
+        if (!valid[i]) continue;
+        uint4 o;
+        if constexpr (OUT == kOutF16) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float a = fabsf(x[i][e]);
+            if (a > 65504.f) {
+              range_hit = true;
+              x[i][e] = copysignf(65504.f, x[i][e]);
+            }
+          }
+          o.x = pack_f16(x[i][0], x[i][1]); o.y = pack_f16(x[i][2], x[i][3]);
+          o.z = pack_f16(x[i][4], x[i][5]); o.w = pack_f16(x[i][6], x[i][7]);
+        } else {
+          o.x = pack_bf16(x[i][0], x[i][1]); o.y = pack_bf16(x[i][2], x[i][3]);
+          o.z = pack_bf16(x[i][4], x[i][5]); o.w = pack_bf16(x[i][6], x[i][7]);
+        }
+        *reinterpret_cast<uint4*>(dst + (row0 + tok[i]) * D + cg * 8) = o;
+      }
+    }
+  }
+  if (range_hit) atomicOr(p.status, JATTN_DEV_RANGE);
+}
+
+// Standalone per-block quantiser of a laid-out [B, H, S, D] 16-bit tensor.
+template <int D, bool IN_BF16>
+__global__ void __launch_bounds__(D / 8 * kTok / kTokPerThread)
+quant_fp8_kernel(const QuantParams p) {
+  constexpr int CG = D / 8;
+  constexpr int NT = CG * kTok / kTokPerThread;
+  constexpr int ROWS_PER_PASS = kTok / kTokPerThread;
+  constexpr int NWARP = NT / 32;
+  __shared__ float red[NWARP];
+  const int tid = threadIdx.x;
+  const int cg = tid % CG, trow = tid / CG;
+  const int blk = blockIdx.x;
+  const size_t bh = blockIdx.y;
+  const uint16_t* x = static_cast<const uint16_t*>(p.x) + bh * p.S * D;
+
+  float v[kTokPerThread][8];
+  bool valid[kTokPerThread];
+  int tok[kTokPerThread];
+  float am = 0.f;
+#pragma unroll
+  for (int i = 0; i < kTokPerThread; ++i) {
+    tok[i] = blk * kTok + trow + i * ROWS_PER_PASS;
+    valid[i] = tok[i] < p.S;
+    uint4 u = valid[i] ? __ldg(reinterpret_cast<const uint4*>(x + static_cast<size_t>(tok[i]) * D + cg * 8))
+                       : make_uint4(0, 0, 0, 0);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if constexpr (IN_BF16) {
+        v[i][2 * e] = __uint_as_float(w[e] << 16);
+        v[i][2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+      } else {
+        __half2 h2 = *reinterpret_cast<const __half2*>(&w[e]);
+        float2 f = __half22float2(h2);
+        v[i][2 * e] = f.x;
+        v[i][2 * e + 1] = f.y;
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(v[i][e]));
+  }
+  am = warp_max(am);
+  if ((tid & 31) == 0) red[tid >> 5] = am;
+  __syncthreads();
+  am = 0.f;
+#pragma unroll
+  for (int w = 0; w < NWARP; ++w) am = fmaxf(am, red[w]);
+  const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+  const float inv = am > 0.f ? __fdiv_rn(448.0f, am) : 1.0f;
+  uint8_t* y = static_cast<uint8_t*>(p.x8) + bh * p.S * D;
+#pragma unroll
+  for (int i = 0; i < kTokPerThread; ++i) {
+    if (!valid[i]) continue;
+    uint2 o;
+    o.x = pack_e4m3x2(__fmul_rn(v[i][0], inv), __fmul_rn(v[i][1], inv)) |
+          (pack_e4m3x2(__fmul_rn(v[i][2], inv), __fmul_rn(v[i][3], inv)) << 16);
+    o.y = pack_e4m3x2(__fmul_rn(v[i][4], inv), __fmul_rn(v[i][5], inv)) |
+          (pack_e4m3x2(__fmul_rn(v[i][6], inv), __fmul_rn(v[i][7], inv)) << 16);
+    *reinterpret_cast<uint2*>(y + static_cast<size_t>(tok[i]) * D + cg * 8) = o;
+  }
+  if (tid == 0) p.scales[bh * p.nblk + blk] = scale;
+}
+
+template <int D, int OUT>
+cudaError_t launch_rope_t(const RopeParams& p, cudaStream_t st) {
+  constexpr int NT = D / 8 * kTok / kTokPerThread;
+  dim3 grid(p.nblk, p.B);
+  rope_qkv_kernel<D, OUT><<<grid, NT, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int D, bool BF>
+cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
+  constexpr int NT = D / 8 * kTok / kTokPerThread;
+  dim3 grid(p.nblk, p.BH);
+  quant_fp8_kernel<D, BF><<<grid, NT, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_rope_qkv(const RopeParams& p, int out_kind, cudaStream_t st) {
+  if (p.d == 128) {
+    if (out_kind == 0) return launch_rope_t<128, kOutF16>(p, st);
+    if (out_kind == 1) return launch_rope_t<128, kOutBF16>(p, st);
+    return launch_rope_t<128, kOutE4M3>(p, st);
+  }
+  if (out_kind == 0) return launch_rope_t<64, kOutF16>(p, st);
+  if (out_kind == 1) return launch_rope_t<64, kOutBF16>(p, st);
+  return launch_rope_t<64, kOutE4M3>(p, st);
+}
+
+cudaError_t launch_quant_fp8(const QuantParams& p, bool in_bf16, cudaStream_t st) {
+  if (p.d == 128) return in_bf16 ? launch_quant_t<128, true>(p, st) : launch_quant_t<128, false>(p, st);
+  return in_bf16 ? launch_quant_t<64, true>(p, st) : launch_quant_t<64, false>(p, st);
+}
+
+}  // namespace jattn

@@ -1,0 +1,254 @@
+"""Python binding of the jattn C ABI (include/jattn.h).
+
+Argument marshalling only: every step of the joint-attention path runs in the
+CUDA kernels of ``libjattn.so``.  PyTorch provides device memory and streams.
+There is no CPU fallback: if the library is missing or no GPU is present the
+calls raise.
+
+Entry points mirror the C names:
+  rope_qkv     joint-sequence assembly + 2D axial RoPE (+ e4m3 quantisation)
+  quant_fp8    per-(b, h, 128-token block) e4m3 quantisation
+  fwd_bf16     attention forward with 16-bit operands, bf16 output
+  fwd_fp8      attention forward with e4m3 operands, bf16 output
+  joint_attention  the whole path in one call (host or device tensors)
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libjattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
+DEV_TIMEOUT, DEV_RANGE = 1, 2
+BF16, FP16, E4M3 = 0, 1, 2
+BLOCK = 128
+
+_DTYPE_CODE = {torch.bfloat16: BF16, torch.float16: FP16, torch.float8_e4m3fn: E4M3}
+_CODE_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, E4M3: torch.float8_e4m3fn}
+_NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
+
+SYMBOLS = ("jattn_rope_qkv", "jattn_quant_fp8", "jattn_fwd_bf16", "jattn_fwd_fp8",
+           "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
+           "jattn_version")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("S_txt", ctypes.c_int32),
+                ("S_img", ctypes.c_int32), ("S_ref", ctypes.c_int32), ("d", ctypes.c_int32)]
+
+
+class JattnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {status_string(code)} (status {code})")
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libjattn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"{path} is missing: run `python -m diffusion_transformer_joint_jattn_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
+    sp = ctypes.POINTER(Shape)
+    lib.jattn_rope_qkv.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), i32, vp, vp, vp, vp, vp]
+    lib.jattn_quant_fp8.argtypes = [sp, i32, vp, vp, vp, vp]
+    lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
+    lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
+    lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
+    lib.jattn_selftest_wait_timeout.argtypes = [i32, vp]
+    lib.jattn_status_string.argtypes = [i32]
+    lib.jattn_status_string.restype = ctypes.c_char_p
+    lib.jattn_version.restype = ctypes.c_char_p
+    for name in SYMBOLS:
+        if name not in ("jattn_status_string", "jattn_version"):
+            getattr(lib, name).restype = i32
+    _lib = lib
+    return lib
+
+
+def status_string(code: int) -> str:
+    return load().jattn_status_string(code).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise JattnError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def make_shape(B, H, S_txt, S_img, S_ref, d) -> Shape:
+    return Shape(B, H, S_txt, S_img, S_ref, d)
+
+
+def n_blocks(S: int) -> int:
+    return -(-S // BLOCK)
+
+
+def rope_qkv(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float = 10000.0,
+             out_dtype="fp16", out=None, stream=None):
+    """Assemble the joint sequence and rotate Q/K.
+
+    qkv_*: bf16 CUDA tensors [B, S_part, 3, H, d] (None for an empty stream);
+    pos: int32 CUDA [S, 3].  Returns (q, k, v, scales); scales is None unless
+    out_dtype is e4m3, then fp32 [3, B, H, ceil(S/128)].
+    """
+    lib = load()
+    parts = [qkv_txt, qkv_img, qkv_ref]
+    ref = next(t for t in parts if t is not None)
+    B, _, _, H, d = ref.shape
+    lens = []
+    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
+        if t is None:
+            lens.append(0)
+            continue
+        _dev(t, name, torch.bfloat16)
+        if t.dim() != 5 or t.shape[0] != B or t.shape[2] != 3 or t.shape[3] != H or t.shape[4] != d:
+            raise ValueError(f"{name} must be [B, S, 3, H, d], got {tuple(t.shape)}")
+        lens.append(t.shape[1])
+    S = sum(lens)
+    _dev(pos, "pos", torch.int32)
+    code = _NAME_CODE[out_dtype] if isinstance(out_dtype, str) else _DTYPE_CODE[out_dtype]
+    odt = _CODE_DTYPE[code]
+    if out is None:
+        dev = ref.device
+        q = torch.empty(B, H, S, d, dtype=odt, device=dev)
+        k = torch.empty_like(q)
+        v = torch.empty_like(q)
+        scales = torch.empty(3, B, H, n_blocks(S), dtype=torch.float32, device=dev) if code == E4M3 else None
+    else:
+        q, k, v, scales = out
+    sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
+    shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
+    _check(lib.jattn_rope_qkv(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
+                              float(theta), sp, code, _ptr(q), _ptr(k), _ptr(v), _ptr(scales), _stream(stream)),
+           "jattn_rope_qkv")
+    return q, k, v, scales
+
+
+def quant_fp8(x: torch.Tensor, out=None, stream=None):
+    """Per-block e4m3 quantisation of a [B, H, S, d] fp16/bf16 tensor."""
+    lib = load()
+    _dev(x, "x")
+    B, H, S, d = x.shape
+    if out is None:
+        x8 = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=x.device)
+        scales = torch.empty(B, H, n_blocks(S), dtype=torch.float32, device=x.device)
+    else:
+        x8, scales = out
+    shape = make_shape(B, H, S, 0, 0, d)
+    _check(lib.jattn_quant_fp8(ctypes.byref(shape), _DTYPE_CODE[x.dtype], _ptr(x), _ptr(x8), _ptr(scales),
+                               _stream(stream)), "jattn_quant_fp8")
+    return x8, scales
+
+
+def _fwd_outputs(B, H, S, d, dev, o, lse, want_lse):
+    if o is None:
+        o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    return o, lse
+
+
+def fwd_bf16(q, k, v, o=None, lse=None, want_lse=False, softmax_scale: float = 0.0, stream=None):
+    """O = softmax(Q K^T * scale) V for fp16/bf16 [B, H, S, d] operands."""
+    lib = load()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev(t, n, q.dtype)
+    B, H, S, d = q.shape
+    o, lse = _fwd_outputs(B, H, S, d, q.device, o, lse, want_lse)
+    shape = make_shape(B, H, S, 0, 0, d)
+    _check(lib.jattn_fwd_bf16(ctypes.byref(shape), _DTYPE_CODE[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o),
+                              _ptr(lse), float(softmax_scale), _stream(stream)), "jattn_fwd_bf16")
+    return o, lse
+
+
+def fwd_fp8(q8, k8, v8, scales, o=None, lse=None, want_lse=False, softmax_scale: float = 0.0, stream=None):
+    """Attention forward on e4m3 [B, H, S, d] operands with fp32 block scales
+    [3, B, H, ceil(S/128)]."""
+    lib = load()
+    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _dev(t, n, torch.float8_e4m3fn)
+    _dev(scales, "scales", torch.float32)
+    B, H, S, d = q8.shape
+    o, lse = _fwd_outputs(B, H, S, d, q8.device, o, lse, want_lse)
+    shape = make_shape(B, H, S, 0, 0, d)
+    _check(lib.jattn_fwd_fp8(ctypes.byref(shape), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(scales), _ptr(o),
+                             _ptr(lse), float(softmax_scale), _stream(stream)), "jattn_fwd_fp8")
+    return o, lse
+
+
+def device_status(clear: bool = True, stream=None):
+    """(status code, raw bits) of the current device's status word."""
+    lib = load()
+    bits = ctypes.c_uint32(0)
+    code = lib.jattn_device_status(_stream(stream), int(clear), ctypes.byref(bits))
+    return code, bits.value
+
+
+def selftest_wait_timeout(limit_ms: int = 50, stream=None):
+    _check(load().jattn_selftest_wait_timeout(int(limit_ms), _stream(stream)), "jattn_selftest_wait_timeout")
+
+
+def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
+                    operand_dtype: str = "fp16", want_lse: bool = False, stream=None):
+    """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8).
+
+    Accepts CUDA tensors, or CPU tensors (then copied to the current device
+    and the output copied back).  Returns O bf16 [B, S, H, d] (and LSE)."""
+    parts = [qkv_txt, qkv_img, qkv_ref]
+    on_host = not next(t for t in parts if t is not None).is_cuda
+    if on_host:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        parts = [None if t is None else t.to(dev, non_blocking=True) for t in parts]
+        pos = pos.to(dev, non_blocking=True)
+    if path == "bf16":
+        q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream)
+        o, lse = fwd_bf16(q, k, v, want_lse=want_lse, stream=stream)
+    elif path == "fp8":
+        q, k, v, sc = rope_qkv(*parts, pos, split, theta, "e4m3", stream=stream)
+        o, lse = fwd_fp8(q, k, v, sc, want_lse=want_lse, stream=stream)
+    else:
+        raise ValueError(f"unknown path {path!r}")
+    if on_host:
+        o = o.to("cpu", non_blocking=False)
+        lse = None if lse is None else lse.to("cpu")
+    return (o, lse) if want_lse else o
+
+
+def flops(B: int, H: int, S: int, d: int) -> int:
+    """Algorithmic FLOPs of one attention call: 4 * B * H * S^2 * d."""
+    return 4 * B * H * S * S * d
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

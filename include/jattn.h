@@ -1,0 +1,161 @@
+/*
+ * jattn -- joint (text + image + reference) DiT attention forward for NVIDIA
+ * B200 (sm_100a), BF16 and FP8 paths.
+ *
+ * The operation ("Speed Up Image Generation with FLUX 3 Image Klein on NVIDIA
+ * Blackwell GPUs"):
+ *   - section "FLUX 3 inference with TensorRT LLM VisualGen": the text, noisy
+ *     target-image and optional reference-image token streams are combined
+ *     through joint attention, i.e. one attention over their concatenation;
+ *   - section "GEMM kernel optimization": rotary position embeddings (RoPE)
+ *     are applied to the query and key projections;
+ *   - section "Quantized and sparse attention": dense BF16 attention and FP8
+ *     attention with FP8 query/key and FP8 value (qk_dtype / v_dtype fp8).
+ * Readings where the page is silent: joint order txt | img | ref with no mask;
+ * 2D axial RoPE over (t, row, col) with per-axis channel spans split[3]
+ * (in that order), interleaved pairs (2p, 2p+1) inside a span of n channels
+ * rotated by pos_axis * theta^(-2p/n); softmax scale 1/sqrt(d); FP8 = e4m3
+ * with one fp32 scale per (batch, head, 128-token block).
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers, 16-byte aligned, row-major and
+ *     contiguous in the layout stated.  The caller allocates and owns every
+ *     buffer; the library allocates nothing and keeps no pointer after the
+ *     call returns.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and the call returns without synchronising.  The host does no
+ *     device synchronisation and no allocation, so the calls can be captured
+ *     into a CUDA graph.
+ *   - Argument errors are reported synchronously, before anything is
+ *     launched: JATTN_ERR_INVALID_ARG (null or inconsistent arguments),
+ *     JATTN_ERR_UNSUPPORTED (d not 64 or 128, dtype not allowed here),
+ *     JATTN_ERR_ALIGNMENT (a pointer not 16-byte aligned).  A failed launch
+ *     returns JATTN_ERR_CUDA.
+ *   - Errors found on the device (a pipeline wait that ran out of time, a
+ *     value out of the 16-bit output range) are recorded in a per-device
+ *     status word; read it with jattn_device_status().  No kernel traps.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef JATTN_H_
+#define JATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  JATTN_OK = 0,
+  JATTN_ERR_INVALID_ARG = 1,
+  JATTN_ERR_UNSUPPORTED = 2,
+  JATTN_ERR_ALIGNMENT = 3,
+  JATTN_ERR_CUDA = 4,
+  JATTN_ERR_TIMEOUT = 5, /* a kernel gave up waiting; see jattn_device_status */
+  JATTN_ERR_RANGE = 6    /* a value exceeded the 16-bit output range (saturated) */
+} jattn_status;
+
+/* Bits of the device status word. */
+#define JATTN_DEV_TIMEOUT 1u
+#define JATTN_DEV_RANGE 2u
+
+typedef enum { JATTN_BF16 = 0, JATTN_FP16 = 1, JATTN_E4M3 = 2 } jattn_dtype;
+
+/* Problem shape.  S = S_txt + S_img + S_ref >= 1, each part >= 0; B, H >= 1;
+ * d in {64, 128}. */
+typedef struct {
+  int32_t B, H, S_txt, S_img, S_ref, d;
+} jattn_shape;
+
+/* Tokens per FP8 scale block (and per attention tile). */
+#define JATTN_BLOCK 128
+
+/*
+ * Joint-sequence assembly + 2D axial RoPE on Q and K (+ optional per-block
+ * e4m3 quantisation), one pass over the inputs.
+ *
+ *   qkv_txt, qkv_img, qkv_ref : bf16 [B, S_part, 3, H, d] (index 0 = Q,
+ *       1 = K, 2 = V) -- the output of each stream's QKV projection.  A part
+ *       with S_part == 0 may be NULL.
+ *   pos    : int32 [S, 3], (t, row, col) of every joint token in the order
+ *            txt | img | ref, shared by all batch entries.
+ *   theta  : RoPE base (> 0), e.g. 10000.
+ *   split  : host array of 3 even, non-negative channel counts for the t, row
+ *            and col axes, summing to d.
+ *   out_dtype:
+ *     JATTN_FP16 / JATTN_BF16 : q, k, v are [B, H, S, d] in that type; q and
+ *        k rotated, v converted.  scales is ignored (may be NULL).  FP16
+ *        values beyond +-65504 are saturated and JATTN_DEV_RANGE is recorded.
+ *     JATTN_E4M3 : q, k, v are e4m3 [B, H, S, d]; scales is fp32
+ *        [3][B][H][ceil(S/128)] (Q, K, V), scale = amax/448 of the block's
+ *        fp32 values (1 for an all-zero block), code = RNE-satfinite
+ *        e4m3(x * (448/amax)).
+ */
+jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                            const void* qkv_ref, const int32_t* pos, float theta,
+                            const int32_t split[3], jattn_dtype out_dtype, void* q, void* k,
+                            void* v, float* scales, void* stream);
+
+/*
+ * Per-block e4m3 quantisation of one laid-out 16-bit tensor.
+ *   x      : in_dtype (JATTN_BF16 or JATTN_FP16) [B, H, S, d]
+ *   x8     : e4m3 [B, H, S, d]
+ *   scales : fp32 [B][H][ceil(S/128)], same arithmetic as jattn_rope_qkv.
+ * Only shape->B, H, d and S = S_txt + S_img + S_ref are used.
+ */
+jattn_status jattn_quant_fp8(const jattn_shape* shape, jattn_dtype in_dtype, const void* x,
+                             void* x8, float* scales, void* stream);
+
+/*
+ * Attention forward, 16-bit operands: O = softmax(Q K^T * softmax_scale) V
+ * over the whole joint sequence (no mask), FP32 accumulation in tensor
+ * memory, online softmax.
+ *   q, k, v : in_dtype (JATTN_FP16 or JATTN_BF16) [B, H, S, d], as written by
+ *             jattn_rope_qkv.
+ *   o       : bf16 [B, S, H, d] (token-major, ready for the output
+ *             projection).
+ *   lse     : fp32 [B, H, S] natural-log sum-exp of the scaled logits, or NULL.
+ *   softmax_scale <= 0 selects 1/sqrt(d).
+ */
+jattn_status jattn_fwd_bf16(const jattn_shape* shape, jattn_dtype in_dtype, const void* q,
+                            const void* k, const void* v, void* o, float* lse,
+                            float softmax_scale, void* stream);
+
+/*
+ * Attention forward, e4m3 operands with per-(b, h, 128-token block) scales:
+ * logits = (q8 . k8) * s_q * s_k, probabilities rounded to e4m3 for the P.V
+ * product, V dequantised by s_v.
+ *   q8, k8, v8 : e4m3 [B, H, S, d] (jattn_rope_qkv with JATTN_E4M3)
+ *   scales     : fp32 [3][B][H][ceil(S/128)]
+ *   o, lse, softmax_scale : as jattn_fwd_bf16.
+ */
+jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void* k8,
+                           const void* v8, const float* scales, void* o, float* lse,
+                           float softmax_scale, void* stream);
+
+/*
+ * Synchronise `stream`, read the current device's status word and return
+ * JATTN_OK, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (timeout wins).  The raw
+ * bits go to *bits if bits is non-NULL.  clear != 0 resets the word.
+ */
+jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits);
+
+/*
+ * Self-test of the bounded waits: one CTA waits on an mbarrier that nothing
+ * arrives on, with a limit of `limit_ms` milliseconds, then records
+ * JATTN_DEV_TIMEOUT and returns.  Used by the failure-detection tests.
+ */
+jattn_status jattn_selftest_wait_timeout(int32_t limit_ms, void* stream);
+
+/* Static description of a status code. */
+const char* jattn_status_string(jattn_status s);
+
+/* Library version, "major.minor.patch". */
+const char* jattn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JATTN_H_ */

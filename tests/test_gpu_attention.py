@@ -1,0 +1,99 @@
+"""GPU parity of the attention forward (jattn_fwd_bf16 / jattn_fwd_fp8) and
+of the whole path (prologue + forward) against the FP64 oracle, through the
+C ABI.
+
+BF16 path (bf16 in, fp16 operands in the MMAs, bf16 out): rel-L2 <= 5e-3 and
+max-abs <= 2e-2 over the sampled rows (all rows for the small cases, 4096
+rows per (b, h) for the large workloads).  The pure-bf16-operand variant is
+checked against its own format floor (see the design notes).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from diffusion_transformer_joint_jattn_b200 import jattn
+from diffusion_transformer_joint_jattn_b200 import workloads as W
+from parity_util import (BF16_MAX_ABS, BF16_REL_L2, gather_lse, gather_rows, max_abs, rel_l2, to_device,
+                         workload_case)
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_bf16(w, inp, dev, operand="fp16", want_lse=True):
+    d = to_device(inp, dev)
+    q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, operand)
+    o, lse = jattn.fwd_bf16(q, k, v, want_lse=want_lse)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+SMALL = [
+    dict(B=1, H=2, d=64, S_txt=32, grid=16, n_ref=0),      # tiny workload, S = 288 (ragged tail)
+    dict(B=1, H=1, d=128, S_txt=1, grid=0, n_ref=0),       # S = 1
+    dict(B=1, H=1, d=128, S_txt=0, grid=16, n_ref=0),      # no text, S = 256 (exact tiles)
+    dict(B=2, H=2, d=128, S_txt=77, grid=9, n_ref=1),      # S = 239, reference image
+    dict(B=1, H=3, d=64, S_txt=3, grid=11, n_ref=0),       # S = 124 < one tile
+    dict(B=1, H=1, d=128, S_txt=129, grid=0, n_ref=0),     # S = 129: one-row tail tile
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"B{c['B']}H{c['H']}d{c['d']}t{c['S_txt']}g{c['grid']}r{c['n_ref']}")
+def test_joint_attention_small_full_rows(cuda_device, case):
+    w = W.custom(**case)
+    inp = W.make_inputs(w, seed=3)
+    o, lse = _run_bf16(w, inp, cuda_device)
+    O, L = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
+    rows = torch.arange(w.S).expand(w.B, w.H, w.S)
+    got = gather_rows(o, rows)
+    assert rel_l2(got, O) <= BF16_REL_L2, rel_l2(got, O)
+    assert max_abs(got, O) <= BF16_MAX_ABS, max_abs(got, O)
+    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=0, atol=2e-3)
+    assert jattn.device_status()[0] == jattn.OK
+
+
+def test_tiny_workload_bf16_operands(cuda_device):
+    """Pure bf16 MMA operands (bf16 rounding of the rotated Q/K and of P):
+    a looser floor set by bf16's 8-bit mantissa, 1e-2 rel-L2."""
+    w = W.BY_NAME["tiny"]
+    inp = W.make_inputs(w, 0)
+    o, _ = _run_bf16(w, inp, cuda_device, operand="bf16")
+    O, _ = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
+    got = gather_rows(o, torch.arange(w.S).expand(w.B, w.H, w.S))
+    assert rel_l2(got, O) <= 1e-2
+
+
+def test_constant_values_through_kernel(cuda_device):
+    """V constant per head -> O equals that constant for every row (checks
+    the P.V product and the normalisation independently of the logits)."""
+    w = W.custom(B=1, H=2, d=128, S_txt=40, grid=15, n_ref=0)        # S = 265
+    inp = W.make_inputs(w, 1)
+    for key in ("qkv_txt", "qkv_img"):
+        inp[key][:, :, 2] = torch.linspace(-2, 2, 128).to(torch.bfloat16)
+    o, _ = _run_bf16(w, inp, cuda_device, want_lse=False)
+    want = torch.linspace(-2, 2, 128).to(torch.bfloat16).to(torch.float32)
+    np.testing.assert_allclose(o.float().cpu().numpy(), np.broadcast_to(want.numpy(), o.shape), atol=2e-2, rtol=0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name", ["t2i_1024_base", "t2i_2048_base", "i2i_2048_base"])
+def test_workload_bf16_sampled_rows(cuda_device, name):
+    w, inp, rows, O, L = workload_case(name)
+    o, lse = _run_bf16(w, inp, cuda_device)
+    got = gather_rows(o, rows)
+    r, m = rel_l2(got, O), max_abs(got, O)
+    print(f"{name}: rel-L2 {r:.3e} max-abs {m:.3e}")
+    assert r <= BF16_REL_L2 and m <= BF16_MAX_ABS
+    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=0, atol=5e-3)
+    assert jattn.device_status()[0] == jattn.OK
+
+
+def test_host_buffers_end_to_end(cuda_device):
+    """The public one-call API with host tensors: copies in, runs the path,
+    copies out; same result as the device-tensor call."""
+    w = W.BY_NAME["tiny"]
+    inp = W.make_inputs(w, 0)
+    o_host = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
+    assert o_host.device.type == "cpu"
+    o_dev, _ = _run_bf16(w, inp, cuda_device, want_lse=False)
+    assert torch.equal(o_host, o_dev.cpu())
