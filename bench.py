@@ -1,0 +1,369 @@
+"""Benchmark: joint-attention TFLOPS on the 2048x2048 Base T2I workload.
+
+One step = one pass of the whole hot path over one batch: jattn_rope_qkv
+(joint-sequence assembly + 2D axial RoPE) followed by jattn_fwd_bf16 (or the
+e4m3 pair for the FP8 path).  TFLOPS = 4 * B * H * S^2 * d / step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Under torchrun each rank runs the same workload on its own GPU with its own
+seed (weak scaling, no data-path collective); the step time is the max over
+ranks.  ``--impl reference`` times the FP64 oracle on the host cores instead
+(rank 0 only), on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from diffusion_transformer_joint_jattn_b200 import workloads as W  # noqa: E402
+
+WORKLOAD = "t2i_2048_base"
+METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
+UNIT = "TFLOPS"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD)
+    ap.add_argument("--no-fp8", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (identity for one rank)."""
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(world: int, flops_per_rank: int, ms_per_step: float) -> float:
+    """Aggregate throughput: every rank processes its own batch (weak
+    scaling), the step takes the slowest rank's time."""
+    return world * flops_per_rank / ms_per_step / 1e9
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank draws its own synthetic batch."""
+    return rank
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def run_ours(args, rank, world, local):
+    from diffusion_transformer_joint_jattn_b200 import jattn
+    import torch.distributed as dist
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    w = W.BY_NAME[args.workload]
+    B, H, S, d = w.B, w.H, w.S, w.d
+    flops = 4 * B * H * S * S * d
+    inp = W.make_inputs(w, seed=rank_seed(rank))
+    dinp = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_ranks(x: float) -> float:
+        return max_over_ranks(x, world, dev)
+
+    def measure(path: str, steps: int, warmup: int):
+        """Time `steps` whole-path steps; events around each kernel."""
+        if path == "bf16":
+            q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
+            bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
+        else:
+            q = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=dev)
+            bufs = (q, torch.empty_like(q), torch.empty_like(q),
+                    torch.empty(3, B, H, jattn.n_blocks(S), dtype=torch.float32, device=dev))
+        o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            if path == "bf16":
+                jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                               "fp16", out=bufs, stream=stream)
+                if ev is not None:
+                    ev[1].record(stream)
+                jattn.fwd_bf16(bufs[0], bufs[1], bufs[2], o=o, stream=stream)
+            else:
+                jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                               "e4m3", out=bufs, stream=stream)
+                if ev is not None:
+                    ev[1].record(stream)
+                jattn.fwd_fp8(bufs[0], bufs[1], bufs[2], bufs[3], o=o, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(warmup):
+            step()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        total_ms = t0.elapsed_time(t1)
+        pro = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
+        fwd = float(np.mean([e[1].elapsed_time(e[2]) for e in evs]))
+        code, bits = jattn.device_status(clear=True)
+        if code != jattn.OK:
+            raise RuntimeError(f"device status {code} bits {bits} after the {path} run")
+        return max_ranks(total_ms / steps), max_ranks(pro), max_ranks(fwd)
+
+    peaks, peak_src = load_peaks()
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms, pro_ms, fwd_ms = measure("bf16", args.steps, args.warmup)
+    clocks = sampler.stop()
+    fp8 = None
+    if not args.no_fp8:
+        ms8, pro8, fwd8 = measure("fp8", args.steps, args.warmup)
+        fp8 = {"value": round(whole_job_tflops(world, flops, ms8), 2), "unit": UNIT, "ms_per_step": round(ms8, 4),
+               "prologue_ms": round(pro8, 4), "fwd_ms": round(fwd8, 4),
+               "roofline": {"bound": "tensor", "achieved": round(flops / fwd8 / 1e9, 2),
+                            "peak": round(2 * peaks["bf16_tflops_sustained"], 1), "unit": "TFLOP/s",
+                            "frac": round(flops / fwd8 / 1e9 / (2 * peaks["bf16_tflops_sustained"]), 4),
+                            "peak_note": f"fp8 = 2 x {peak_src} bf16 sustained (nominal fp8/bf16 ratio)",
+                            "frac_of_nominal_4500": round(flops / fwd8 / 1e9 / 4500.0, 4), "traffic": None}}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(jattn, w, inp, dev, stream, min(args.steps, 10), 2, flops, world, max_ranks, barrier)
+
+    achieved = flops / fwd_ms / 1e9
+    peak = peaks["bf16_tflops_sustained"]
+    line = {
+        "metric": METRIC, "value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "S": S, "S_txt": w.S_txt, "S_img": w.S_img,
+                   "S_ref": w.S_ref, "d": d, "rope_split": list(w.split), "theta": w.theta,
+                   "path": "bf16 in/out, fp16 MMA operands, fp32 accumulate",
+                   "l2": "inputs larger than L2 (623 MB qkv streams, 622 MB laid-out q/k/v)",
+                   "parallelism": f"replicas x{world}"},
+        "prologue_ms": round(pro_ms, 4), "fwd_ms": round(fwd_ms, 4),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(achieved / peak, 4),
+                     "peak_note": f"{peak_src} cuBLAS bf16 sustained (MEASURED_PEAKS.json bf16_tflops_sustained)",
+                     "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
+                     "frac_of_nominal_2250": round(achieved / 2250.0, 4),
+                     "traffic": None,
+                     "kernel": "attn_fwd_kernel<128,false>"},
+        "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / pro_ms / 1e6, 1),
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(prologue_bytes(w, 2) / pro_ms / 1e6 / peaks["hbm_gbs"], 4)},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if fp8 is not None:
+        line["fp8"] = fp8
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, target_s=12.0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def prologue_bytes(w, out_bytes: int) -> int:
+    """Algorithmic bytes of one prologue call: read 3*B*S*H*d bf16, write the
+    same count in the output type (+ scales, negligible)."""
+    n = 3 * w.B * w.S * w.H * w.d
+    return n * 2 + n * out_bytes
+
+
+def measure_e2e(jattn, w, inp, dev, stream, steps, warmup, flops, world, max_over_ranks, barrier):
+    """Public one-call API with host (pinned) buffers: H2D of the step's
+    inputs, the path, D2H of the output, all inside the timed region."""
+    host = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
+    out_host = torch.empty(w.B, w.S, w.H, w.d, dtype=torch.bfloat16).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+    d2h = out_host.numel() * out_host.element_size()
+
+    def one():
+        jattn.joint_attention(host["qkv_txt"], host["qkv_img"], host["qkv_ref"], host["pos"], w.split, w.theta,
+                              out=out_host)
+
+    for _ in range(warmup):
+        one()
+    barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(steps):
+        one()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1) / steps)
+    return {"value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "api": "jattn.joint_attention (pinned host in/out)"}
+
+
+def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
+    """Run the FP64 oracle on `heads` (b, h) pairs x `rows_per_head` query
+    rows of workload w.  Returns (seconds, flops)."""
+    import oracle
+    sub = w.with_batch_heads(B=1, H=heads)
+    inp = W.make_inputs(sub, seed)
+    rows = W.sample_rows(sub, rows_per_head, seed)
+    workers = max(1, (os.cpu_count() or 2) // 2)
+    t = time.perf_counter()
+    oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], sub.split, sub.theta,
+                           rows=rows, workers=workers)
+    dt = time.perf_counter() - t
+    return dt, 4 * heads * rows.shape[-1] * w.S * w.d, workers
+
+
+def cpu_baseline(w, target_s: float = 12.0):
+    # calibrate on a small sample, then size the sample for ~target_s seconds
+    dt, fl, _ = oracle_sample(w, 128, 2)
+    rate = fl / dt
+    heads = 8
+    rows = int(max(128, min(w.S, target_s * rate / (4 * heads * w.S * w.d))))
+    dt, fl, workers = oracle_sample(w, rows, heads)
+    return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": os.cpu_count(), "threads": workers,
+            "kind": "oracle",
+            "sample": f"{heads} heads x {rows} sampled query rows of {w.name} (S={w.S}, d={w.d}), "
+                      f"FP64 numpy oracle incl. RoPE, {dt:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    w = W.BY_NAME[args.workload]
+    flops = 4 * w.B * w.H * w.S * w.S * w.d
+    dt, fl, workers = oracle_sample(w, 128, 2)
+    rate = fl / dt
+    steps_budget_s = 150.0
+    per_step_s = max(1.0, steps_budget_s / max(1, args.steps + args.warmup))
+    rows = int(max(32, min(w.S, per_step_s * rate / (4 * 2 * w.S * w.d))))
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, fl, workers = oracle_sample(w, rows, 2, seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+    sec = float(np.mean(times))
+    value = fl / sec / 1e12
+    ms_full = flops / (fl / sec) * 1e3
+    line = {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_full, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "d": w.d,
+                       "note": "each step = FP64 oracle on 2 heads x %d sampled rows; ms_per_step extrapolated "
+                               "to the full call from the sampled rate" % rows},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": os.cpu_count(), "threads": workers,
+                             "kind": "oracle", "sample": f"2 heads x {rows} query rows per step"},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

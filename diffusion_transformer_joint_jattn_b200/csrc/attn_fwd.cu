@@ -107,6 +107,10 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
   uint16_t lo, hi;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(b), "f"(a));
@@ -114,10 +118,13 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
-template <int D, bool FP8>
+// KIND: 0 = fp16 operands, 1 = bf16 operands, 2 = e4m3 operands.
+template <int D, int KIND>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const FwdParams p, const uint32_t in_fmt) {
+                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  constexpr bool FP8 = KIND == 2;
+  constexpr uint32_t in_fmt = KIND == 1 ? 1u : 0u;   // f16 / bf16 (kind::f16); e4m3 (kind::f8f6f4)
   using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms.
@@ -276,7 +283,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
     // exceeds the e4m3 range while p <= 2^8.
-    const float p8_log2 = 2.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
+    const float p8_log2 = 8.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
 
     for (int j = 0; j < n_kv; ++j) {
       const int sb = j & 1;
@@ -341,7 +348,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const float p0 = ex2_approx(fmaf(v[2 * c + 0], c_j, neg_m));
           const float p1 = ex2_approx(fmaf(v[2 * c + 1], c_j, neg_m));
           ls += p0 + p1;
-          pk[c] = pack_f16x2(p0, p1);
+          pk[c] = KIND == 1 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
         }
       }
       l_run += ls;
@@ -418,16 +425,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
-template <int D, bool FP8>
-cudaError_t launch_t(const FwdParams& p, uint32_t in_fmt, const CUtensorMap& tq, const CUtensorMap& tk,
-                     const CUtensorMap& tv, cudaStream_t st) {
-  using C = Cfg<D, FP8>;
+template <int D, int KIND>
+cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                     cudaStream_t st) {
+  using C = Cfg<D, KIND == 2>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  auto kern = attn_fwd_kernel<D, FP8>;
+  auto kern = attn_fwd_kernel<D, KIND>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_tiles, p.B * p.H);
-  kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, p, in_fmt);
+  kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
 
@@ -450,13 +457,13 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
 
 cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  const uint32_t fmt = in_bf16 ? 1u : 0u;
-  return d == 128 ? launch_t<128, false>(p, fmt, tq, tk, tv, st) : launch_t<64, false>(p, fmt, tq, tk, tv, st);
+  if (in_bf16) return d == 128 ? launch_t<128, 1>(p, tq, tk, tv, st) : launch_t<64, 1>(p, tq, tk, tv, st);
+  return d == 128 ? launch_t<128, 0>(p, tq, tk, tv, st) : launch_t<64, 0>(p, tq, tk, tv, st);
 }
 
 cudaError_t launch_fwd_fp8(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, cudaStream_t st) {
-  return d == 128 ? launch_t<128, true>(p, 0u, tq, tk, tv, st) : launch_t<64, true>(p, 0u, tq, tk, tv, st);
+  return d == 128 ? launch_t<128, 2>(p, tq, tk, tv, st) : launch_t<64, 2>(p, tq, tk, tv, st);
 }
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st) {

@@ -220,11 +220,13 @@ def selftest_wait_timeout(limit_ms: int = 50, stream=None):
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
-                    operand_dtype: str = "fp16", want_lse: bool = False, stream=None):
+                    operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None):
     """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8).
 
     Accepts CUDA tensors, or CPU tensors (then copied to the current device
-    and the output copied back).  Returns O bf16 [B, S, H, d] (and LSE)."""
+    -- asynchronously when they are pinned -- and the output copied back,
+    into ``out`` if given, e.g. a pinned bf16 [B, S, H, d] buffer).
+    Returns O bf16 [B, S, H, d] (and LSE)."""
     parts = [qkv_txt, qkv_img, qkv_ref]
     on_host = not next(t for t in parts if t is not None).is_cuda
     if on_host:
@@ -240,7 +242,13 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
     else:
         raise ValueError(f"unknown path {path!r}")
     if on_host:
-        o = o.to("cpu", non_blocking=False)
+        if out is not None:
+            out.copy_(o, non_blocking=out.is_pinned())
+            if out.is_pinned():
+                torch.cuda.current_stream().synchronize()
+            o = out
+        else:
+            o = o.to("cpu")
         lse = None if lse is None else lse.to("cpu")
     return (o, lse) if want_lse else o
 

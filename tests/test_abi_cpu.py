@@ -1,0 +1,101 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/jattn.h declares, and rejects invalid arguments synchronously with
+the documented status codes (before touching the device).  No call here
+reaches a kernel launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from diffusion_transformer_joint_jattn_b200 import jattn
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "jattn.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(jattn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("jattn_rope_qkv", "jattn_quant_fp8", "jattn_fwd_bf16", "jattn_fwd_fp8"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = jattn.load()
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version():
+    assert jattn.status_string(jattn.OK) == "ok"
+    assert "aligned" in jattn.status_string(jattn.ERR_ALIGNMENT)
+    assert jattn.load().jattn_version().decode().count(".") == 2
+
+
+A = 1 << 20          # a 16-byte aligned fake address: never dereferenced (validation fails first)
+
+
+def shape(B=1, H=1, St=10, Si=0, Sr=0, d=128):
+    return ctypes.byref(jattn.make_shape(B, H, St, Si, Sr, d))
+
+
+@pytest.mark.parametrize("args,code", [
+    (dict(St=0), jattn.ERR_INVALID_ARG),                 # S = 0
+    (dict(B=0), jattn.ERR_INVALID_ARG),
+    (dict(St=-1, Si=5), jattn.ERR_INVALID_ARG),
+    (dict(d=96), jattn.ERR_UNSUPPORTED),
+    (dict(d=256), jattn.ERR_UNSUPPORTED),
+    (dict(B=300, H=300), jattn.ERR_INVALID_ARG),         # B*H beyond the grid limit
+])
+def test_fwd_rejects_bad_shapes(args, code):
+    lib = jattn.load()
+    assert lib.jattn_fwd_bf16(shape(**args), jattn.FP16, A, A, A, A, None, 0.0, None) == code
+
+
+def test_fwd_rejects_bad_pointers_and_dtypes():
+    lib = jattn.load()
+    assert lib.jattn_fwd_bf16(shape(), jattn.FP16, None, A, A, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
+    assert lib.jattn_fwd_bf16(shape(), jattn.FP16, A + 8, A, A, A, None, 0.0, None) == jattn.ERR_ALIGNMENT
+    assert lib.jattn_fwd_bf16(shape(), jattn.FP16, A, A, A, A + 2, None, 0.0, None) == jattn.ERR_ALIGNMENT
+    assert lib.jattn_fwd_bf16(shape(), jattn.E4M3, A, A, A, A, None, 0.0, None) == jattn.ERR_UNSUPPORTED
+    assert lib.jattn_fwd_bf16(shape(), jattn.FP16, A, A, A, A, A + 1, 0.0, None) == jattn.ERR_ALIGNMENT
+    assert lib.jattn_fwd_bf16(shape(), jattn.FP16, A, A, A, A, None, float("nan"), None) == jattn.ERR_INVALID_ARG
+    assert lib.jattn_fwd_fp8(shape(), A, A, A, None, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
+
+
+def _split(*v):
+    return (ctypes.c_int32 * 3)(*v)
+
+
+def test_rope_rejects_bad_arguments():
+    lib = jattn.load()
+    ok_split = _split(16, 56, 56)
+    f = lib.jattn_rope_qkv
+    # split must be even, non-negative and sum to d
+    assert f(shape(), A, None, None, A, 1e4, _split(16, 56, 58), jattn.FP16, A, A, A, None, None) == jattn.ERR_INVALID_ARG
+    assert f(shape(), A, None, None, A, 1e4, _split(15, 57, 56), jattn.FP16, A, A, A, None, None) == jattn.ERR_INVALID_ARG
+    # a non-empty stream needs a pointer; theta must be positive
+    assert f(shape(Si=4), A, None, None, A, 1e4, ok_split, jattn.FP16, A, A, A, None, None) == jattn.ERR_INVALID_ARG
+    assert f(shape(), A, None, None, A, -1.0, ok_split, jattn.FP16, A, A, A, None, None) == jattn.ERR_INVALID_ARG
+    # e4m3 output needs a scales buffer
+    assert f(shape(), A, None, None, A, 1e4, ok_split, jattn.E4M3, A, A, A, None, None) == jattn.ERR_INVALID_ARG
+    # alignment of a stream and of an output
+    assert f(shape(), A + 4, None, None, A, 1e4, ok_split, jattn.FP16, A, A, A, None, None) == jattn.ERR_ALIGNMENT
+    assert f(shape(), A, None, None, A, 1e4, ok_split, jattn.FP16, A, A + 8, A, None, None) == jattn.ERR_ALIGNMENT
+    assert f(shape(), A, None, None, A, 1e4, ok_split, 7, A, A, A, None, None) == jattn.ERR_UNSUPPORTED
+
+
+def test_quant_rejects_bad_arguments():
+    lib = jattn.load()
+    f = lib.jattn_quant_fp8
+    assert f(shape(), jattn.E4M3, A, A, A, None) == jattn.ERR_UNSUPPORTED
+    assert f(shape(), jattn.FP16, A, A, None, None) == jattn.ERR_INVALID_ARG
+    assert f(shape(), jattn.FP16, A + 2, A, A, None) == jattn.ERR_ALIGNMENT
+
+
+def test_selftest_rejects_bad_limit():
+    assert jattn.load().jattn_selftest_wait_timeout(0, None) == jattn.ERR_INVALID_ARG

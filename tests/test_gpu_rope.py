@@ -1,9 +1,11 @@
 """GPU parity of the prologue (jattn_rope_qkv, jattn_quant_fp8) against the
 oracle, through the C ABI.
 
-* 16-bit outputs: every element within 1 unit in the last place of the
-  oracle's FP64 rotation rounded to the same type (the kernel rotates in
-  fp32); V exactly equal (a conversion).
+* 16-bit outputs: every element within half a unit in the last place of the
+  oracle's FP64 rotation plus the fp32 rotation error bound (a few fp32 ulps
+  of the pair's magnitude, which matters only under cancellation), and at
+  least 99% of them equal to the exactly rounded value; V exactly equal (a
+  conversion).
 * e4m3 outputs: codes equal to the oracle's encoding of the same values,
   except where the value sits within 2^-20 of an e4m3 rounding midpoint
   (there an fp32-vs-fp64 last-bit difference may flip the code by one step);
@@ -22,14 +24,23 @@ from parity_util import to_device
 pytestmark = pytest.mark.gpu
 
 
-def _ulp_diff_16(a: torch.Tensor, b: torch.Tensor) -> np.ndarray:
-    """|a - b| in units of the last place of the 16-bit type (same sign)."""
-    ia = a.contiguous().view(torch.int16).to(torch.int64).numpy()
-    ib = b.contiguous().view(torch.int16).to(torch.int64).numpy()
-    # map sign-magnitude to a monotonic integer line
-    ia = np.where(ia < 0, -(ia & 0x7FFF), ia)
-    ib = np.where(ib < 0, -(ib & 0x7FFF), ib)
-    return np.abs(ia - ib)
+def _ulp16(y: np.ndarray, dtype) -> np.ndarray:
+    mant = 10 if dtype == torch.float16 else 7
+    emin = -14 if dtype == torch.float16 else -126
+    e = np.floor(np.log2(np.maximum(np.abs(y), 2.0 ** emin)))
+    return 2.0 ** (e - mant)
+
+
+def _check_rotated(got: torch.Tensor, ref: np.ndarray, dtype, name: str):
+    """got: 16-bit [..., d]; ref: float64 exact rotation [..., d]."""
+    g = got.cpu().to(torch.float64).numpy()
+    pair = np.sqrt(ref[..., 0::2] ** 2 + ref[..., 1::2] ** 2)
+    pair = np.repeat(pair, 2, axis=-1)
+    bound = 0.5 * _ulp16(ref, dtype) * (1 + 2.0 ** -10) + 2.0 ** -20 * pair
+    err = np.abs(g - ref)
+    assert np.all(err <= bound), f"{name}: {np.sum(err > bound)} elements beyond the bound, worst {np.max(err / bound):.2f}x"
+    exact = torch.from_numpy(ref).to(dtype).to(torch.float64).numpy()
+    assert np.mean(g != exact) < 0.01, f"{name}: {100 * np.mean(g != exact):.3f}% not exactly rounded"
 
 
 def _expected_rot(w, inp):
@@ -58,10 +69,7 @@ def test_rope_16bit_within_one_ulp(cuda_device, case, out):
     qr, kr, vr = _expected_rot(w, inp)
     dt = torch.float16 if out == "fp16" else torch.bfloat16
     for name, got, ref in (("q", q, qr), ("k", k, kr)):
-        want = torch.from_numpy(ref).to(dt)
-        diff = _ulp_diff_16(got.cpu(), want)
-        assert diff.max() <= 1, f"{name}: max ulp diff {diff.max()}"
-        assert (diff > 0).mean() < 0.01, f"{name}: {100 * (diff > 0).mean():.3f}% off by one ulp"
+        _check_rotated(got, ref, dt, name)
     assert torch.equal(v.cpu(), torch.from_numpy(vr).to(dt))
     code, bits = jattn.device_status()
     assert code == jattn.OK and bits == 0
@@ -136,9 +144,7 @@ def test_rope_full_size_2048(cuda_device):
         pos = inp["pos"][toks].numpy()
         for which, got in ((0, q), (1, k)):
             xr = oracle.rope_rotate(np.transpose(x[:, which], (1, 0, 2)), pos, w.split, w.theta)
-            want = torch.from_numpy(xr).to(torch.float16)
-            diff = _ulp_diff_16(got[b][:, toks].cpu(), want)
-            assert diff.max() <= 1
+            _check_rotated(got[b][:, toks], xr, torch.float16, "qk"[which])
     # full-tensor scale check on V (exact) and Q (rel 1e-6)
     vr = qkv[..., 2, :, :].permute(0, 2, 1, 3).to(torch.float32).numpy()
     _, sv = oracle.quantize_blocks(vr)
