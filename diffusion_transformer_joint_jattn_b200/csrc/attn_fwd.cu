@@ -7,16 +7,25 @@
 // path with FP8 query/key and FP8 value.  The page names library kernels only;
 // this kernel is written for B200 from the definition.
 //
-// One CTA computes one 128-row query tile of one (batch, head):
-//   warp 4      TMA producer: Q once, then K_j and V_j tiles into smem rings
-//   warp 5      MMA issuer (one thread): S_j = Q K_j^T into TMEM (two S
-//               buffers), then O += P_{j-1} V_{j-1} with P read from TMEM
-//   warps 0..3  softmax: one thread per query row (= TMEM lane); online
-//               softmax with a lazy rescale (O and l are rescaled only when
-//               the running max grows by more than 2^8), P written back to
-//               TMEM as fp16 / e4m3; epilogue O / l -> bf16 [B, S, H, d].
-// Accumulators live in TMEM: S0 [0,128), S1 [128,256), O [256, 256+d),
-// P [384, 448).  Every wait is bounded (see ptx_sm100.cuh).
+// One CTA computes two 128-row query tiles (t = 0, 1) of one (batch, head):
+//   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one thread
+//               per query row (= TMEM lane), online softmax with a lazy
+//               rescale (O and l are rescaled only when the running max grows
+//               by more than 2^8), P written back into the tile's S columns;
+//               epilogue O / l -> bf16 [B, S, H, d].
+//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j.
+//               Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): each
+//               tile's softmax overlaps the other tile's tensor work.
+//   warp 9      TMA producer: Q tiles once, K_j / V_j into smem rings.
+//   (warps 10, 11 idle: they complete the third warpgroup.)
+// The block starts at 168 registers per thread (384 x 168 = 64512); the
+// MMA/TMA warpgroup then releases registers down to 56 and the two softmax
+// warpgroups grow to 224 (2 x 128 x 224 + 128 x 56 = 64512).
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256, 256+d), O_1 [384, 384+d).
+// Because the tensor pipe runs one thread's MMAs in order, the commit that
+// signals S_t(j) also proves PV_t(j-1) finished: O_t is stable for the
+// rescale, and P_t(j-1) has been consumed before S_t(j) overwrites it.
+// Every wait is bounded (see ptx_sm100.cuh).
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -28,14 +37,20 @@ namespace jattn {
 
 namespace {
 
-constexpr int BM = 128;              // query rows per CTA
+constexpr int BM = 128;              // query rows per tile
+constexpr int NQ = 2;                // query tiles per CTA
 constexpr int BN = 128;              // keys per tile
-constexpr int kThreads = 192;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
+constexpr int kMmaWarp = 8;
+constexpr int kProducerWarp = 9;
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsSoftmax = 224;
+constexpr uint32_t kRegsOther = 56;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: P <= 2^8 before rescale
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: P <= 2^8 before a rescale
+
+__host__ __device__ constexpr uint32_t col_s(int t) { return static_cast<uint32_t>(t) * 128u; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
 
 template <int D, bool FP8>
 struct Cfg {
@@ -50,18 +65,16 @@ struct Cfg {
   static constexpr int MK = FP8 ? 32 : 16;            // K per MMA instruction
   static constexpr int QK_STEPS = RB / 32;            // 32 bytes of K per step
   static constexpr int PV_STEPS = BN / MK;
-  static constexpr int STAGES = (TB >= 32768) ? 3 : 4;
-  static constexpr int SMEM = (1 + 2 * STAGES) * TB + 2048;
-  static constexpr int P_COLS = BN * (FP8 ? 1 : 2) / 4;
+  static constexpr int KS = TB >= 32768 ? 3 : 4;      // K ring stages
+  static constexpr int VS = TB >= 32768 ? 2 : 4;      // V ring stages
+  static constexpr int SMEM = (NQ + KS + VS) * TB + 2048;
 };
 
 struct __align__(8) Bars {
   uint64_t q_full;
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
-  uint64_t s_full[2], s_empty[2];
-  uint64_t p_full;
-  uint64_t o_done;
+  uint64_t s_full[NQ], p_full[NQ], o_final[NQ];
   uint64_t mma_final;
   uint32_t tmem_base;
   uint32_t abort;
@@ -117,6 +130,11 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 
 // KIND: 0 = fp16 operands, 1 = bf16 operands, 2 = e4m3 operands.
 template <int D, int KIND>
@@ -127,35 +145,36 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   constexpr uint32_t in_fmt = KIND == 1 ? 1u : 0u;   // f16 / bf16 (kind::f16); e4m3 (kind::f8f6f4)
   using C = Cfg<D, FP8>;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte alignment for the 128-byte swizzle atoms.
+  // 1024-byte alignment for the swizzle atoms.
   const uint32_t raw_u32 = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw_u32 & 1023u)) & 1023u);
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + C::TB;
-  uint8_t* sV = sK + C::STAGES * C::TB;
-  Bars* bar = reinterpret_cast<Bars*>(sV + C::STAGES * C::TB);
+  uint8_t* sQ = smem;                                  // NQ tiles
+  uint8_t* sK = sQ + NQ * C::TB;
+  uint8_t* sV = sK + C::KS * C::TB;
+  Bars* bar = reinterpret_cast<Bars*>(sV + C::VS * C::TB);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qt = blockIdx.x;
+  const int qp = blockIdx.x;                           // pair of query tiles
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
   const int n_kv = p.n_tiles;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar->q_full, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KS; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::VS; ++s) {
       mbar_init(&bar->v_full[s], 1);
       mbar_init(&bar->v_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar->s_full[s], 1);
-      mbar_init(&bar->s_empty[s], BM);
+    for (int t = 0; t < NQ; ++t) {
+      mbar_init(&bar->s_full[t], 1);
+      mbar_init(&bar->p_full[t], BM);
+      mbar_init(&bar->o_final[t], 1);
     }
-    mbar_init(&bar->p_full, BM);
-    mbar_init(&bar->o_done, 1);
     mbar_init(&bar->mma_final, 1);
     bar->abort = 0;
     fence_mbarrier_init();
@@ -170,98 +189,118 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = bar->tmem_base;
   const WaitCtl ctl{&bar->abort, p.status, p.timeout_ns};
-
-  if (warp == kProducerWarp) {
+  if (warp >= 8) {
+    // Third warpgroup: producer, MMA issuer and two idle warps.
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar->q_full, C::TB);
-      for (int x = 0; x < C::NBOX; ++x)
-        tma_load_3d(&tmQ, &bar->q_full, sQ + x * C::BOXB, x * C::BOX_ELEMS, qt * BM, bh);
-      int issued = 0;
+      mbar_arrive_expect_tx(&bar->q_full, NQ * C::TB);
+      for (int t = 0; t < NQ; ++t)
+        for (int x = 0; x < C::NBOX; ++x)
+          tma_load_3d(&tmQ, &bar->q_full, sQ + t * C::TB + x * C::BOXB, x * C::BOX_ELEMS, (qp * NQ + t) * BM, bh);
+      int nk = 0, nv = 0;
       for (int j = 0; j < n_kv; ++j) {
-        const int s = j % C::STAGES;
-        const uint32_t ph = ((j / C::STAGES) & 1) ^ 1;
-        if (!mbar_wait(&bar->k_empty[s], ph, ctl)) break;
-        mbar_arrive_expect_tx(&bar->k_full[s], C::TB);
+        const int ks = j % C::KS;
+        if (!mbar_wait(&bar->k_empty[ks], ((j / C::KS) & 1) ^ 1, ctl)) break;
+        mbar_arrive_expect_tx(&bar->k_full[ks], C::TB);
         for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmK, &bar->k_full[s], sK + s * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
-        if (!mbar_wait(&bar->v_empty[s], ph, ctl)) { issued = 2 * j + 1; break; }
-        mbar_arrive_expect_tx(&bar->v_full[s], C::TB);
+          tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
+        nk = j + 1;
+        const int vs = j % C::VS;
+        if (!mbar_wait(&bar->v_empty[vs], ((j / C::VS) & 1) ^ 1, ctl)) break;
+        mbar_arrive_expect_tx(&bar->v_full[vs], C::TB);
         for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmV, &bar->v_full[s], sV + s * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
-        issued = 2 * j + 2;
+          tma_load_3d(&tmV, &bar->v_full[vs], sV + vs * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
+        nv = j + 1;
       }
       // Drain: every load issued must have landed before the CTA may exit.
       drain_wait(&bar->q_full, 0, ctl);
-      const int nk = (issued + 1) / 2, nv = issued / 2;
-      for (int s = 0; s < C::STAGES; ++s) {
-        if (s < nk) drain_wait(&bar->k_full[s], ((nk - 1 - s) / C::STAGES) & 1, ctl);
-        if (s < nv) drain_wait(&bar->v_full[s], ((nv - 1 - s) / C::STAGES) & 1, ctl);
-      }
+      for (int s = 0; s < C::KS && s < nk; ++s) drain_wait(&bar->k_full[s], ((nk - 1 - s) / C::KS) & 1, ctl);
+      for (int s = 0; s < C::VS && s < nv; ++s) drain_wait(&bar->v_full[s], ((nv - 1 - s) / C::VS) & 1, ctl);
     }
-  } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc_qk = instr_desc(in_fmt, in_fmt, 0, BM, BN);
       const uint32_t idesc_pv = instr_desc(in_fmt, in_fmt, 1, BM, D);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
-      bool ok = mbar_wait(&bar->q_full, 0, ctl);
       bool any_mma = false;
-      auto issue_pv = [&](int i) -> bool {
-        const int s = i % C::STAGES;
-        if (!mbar_wait(&bar->p_full, i & 1, ctl)) return false;
-        if (!mbar_wait(&bar->v_full[s], (i / C::STAGES) & 1, ctl)) return false;
-        tc_fence_after();
-        const uint32_t vbase = sVa + s * C::TB;
+      auto issue_qk = [&](int t, int ks) {
+        const uint32_t kbase = sKa + ks * C::TB;
+        const uint32_t qbase = sQa + t * C::TB;
+#pragma unroll
+        for (int kk = 0; kk < C::QK_STEPS; ++kk) {
+          const uint32_t off = (kk * 32) / C::SWB * C::BOXB + (kk * 32) % C::SWB;
+          const uint64_t adesc = smem_desc(qbase + off, 16, 8 * C::SWB, C::SWMODE);
+          const uint64_t bdesc = smem_desc(kbase + off, 16, 8 * C::SWB, C::SWMODE);
+          if constexpr (FP8) mma_f8_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, kk > 0);
+          else mma_f16_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, kk > 0);
+        }
+        any_mma = true;
+      };
+      auto issue_pv = [&](int t, int vs, bool acc) {
+        const uint32_t vbase = sVa + vs * C::TB;
 #pragma unroll
         for (int kk = 0; kk < C::PV_STEPS; ++kk) {
           const uint64_t bdesc = smem_desc(vbase + kk * C::MK * C::SWB, C::BOXB, 8 * C::SWB, C::SWMODE);
-          if constexpr (FP8) mma_f8_ts(tmem + kColO, tmem + kColP + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0));
-          else mma_f16_ts(tmem + kColO, tmem + kColP + kk * 8, bdesc, idesc_pv, (i > 0 || kk > 0));
+          if constexpr (FP8) mma_f8_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, acc || kk > 0);
+          else mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, acc || kk > 0);
         }
-        mma_commit(&bar->v_empty[s]);
-        mma_commit(&bar->o_done);
-        return true;
       };
+      bool ok = mbar_wait(&bar->q_full, 0, ctl) && mbar_wait(&bar->k_full[0], 0, ctl);
       if (ok) {
         tc_fence_after();
-        for (int j = 0; j < n_kv && ok; ++j) {
-          const int s = j % C::STAGES, sb = j & 1;
-          ok = mbar_wait(&bar->k_full[s], (j / C::STAGES) & 1, ctl) &&
-               mbar_wait(&bar->s_empty[sb], ((j >> 1) & 1) ^ 1, ctl);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t kbase = sKa + s * C::TB;
-          const uint32_t d_s = tmem + (sb ? kColS1 : kColS0);
-#pragma unroll
-          for (int kk = 0; kk < C::QK_STEPS; ++kk) {
-            const uint32_t off = (kk * 32) / C::SWB * C::BOXB + (kk * 32) % C::SWB;
-            const uint64_t adesc = smem_desc(sQa + off, 16, 8 * C::SWB, C::SWMODE);
-            const uint64_t bdesc = smem_desc(kbase + off, 16, 8 * C::SWB, C::SWMODE);
-            if constexpr (FP8) mma_f8_ss(d_s, adesc, bdesc, idesc_qk, kk > 0);
-            else mma_f16_ss(d_s, adesc, bdesc, idesc_qk, kk > 0);
-          }
-          any_mma = true;
-          mma_commit(&bar->s_full[sb]);
-          mma_commit(&bar->k_empty[s]);
-          if (j > 0) ok = issue_pv(j - 1);
+        for (int t = 0; t < NQ; ++t) {
+          issue_qk(t, 0);
+          mma_commit(&bar->s_full[t]);
         }
-        if (ok) issue_pv(n_kv - 1);
+        mma_commit(&bar->k_empty[0]);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int vs = j % C::VS;
+          const int ks = (j + 1) % C::KS;
+          const bool more = j + 1 < n_kv;
+          ok = mbar_wait(&bar->v_full[vs], (j / C::VS) & 1, ctl);
+          for (int t = 0; t < NQ && ok; ++t) {
+            ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, vs, j > 0);
+            if (t == NQ - 1) mma_commit(&bar->v_empty[vs]);
+            if (more) {
+              if (t == 0) {
+                ok = mbar_wait(&bar->k_full[ks], ((j + 1) / C::KS) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
+              }
+              issue_qk(t, ks);
+              mma_commit(&bar->s_full[t]);
+              if (t == NQ - 1) mma_commit(&bar->k_empty[ks]);
+            } else {
+              mma_commit(&bar->o_final[t]);
+            }
+          }
+        }
       }
       if (any_mma) {
         mma_commit(&bar->mma_final);
         drain_wait(&bar->mma_final, 0, ctl);
       }
     }
+    }
   } else {
     // ------------------------------------------------------------ softmax
-    const int row = warp * 32 + lane;                 // TMEM lane == query row
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    const int t = warp >> 2;                          // query tile of this warpgroup
+    const int row = (warp & 3) * 32 + lane;           // TMEM lane == row in the tile
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t ts = tmem + lane_base + col_s(t);
+    const uint32_t to = tmem + lane_base + col_o(t);
     const float sl2 = p.scale_log2;
-    const int q_row = qt * BM + row;
+    const int q_row = (qp * NQ + t) * BM + row;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
 
@@ -272,7 +311,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const size_t nb = static_cast<size_t>(p.n_tiles);
       const size_t bhn = static_cast<size_t>(bh) * nb;
       const size_t plane = static_cast<size_t>(p.B) * p.H * nb;
-      sq = p.scales[bhn + qt];
+      sq = p.scales[bhn + min(qp * NQ + t, p.n_tiles - 1)];
       sc_k = p.scales + plane + bhn;
       sc_v = p.scales + 2 * plane + bhn;
       float mv = 0.f;
@@ -286,24 +325,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float p8_log2 = 8.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
 
     for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      ok = warp_wait(&bar->s_full[sb], (j >> 1) & 1, ctl);
+      ok = warp_wait(&bar->s_full[t], j & 1, ctl);
       if (!ok) break;
       __syncwarp();
       tc_fence_after();
       float v[BN];
-      {
+#pragma unroll
+      for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        const uint32_t ts = tmem + lane_base + (sb ? kColS1 : kColS0);
+        tmem_ld32(ts + c * 32, r);
 #pragma unroll
-        for (int c = 0; c < BN / 32; ++c) {
-          tmem_ld32(ts + c * 32, r);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) v[c * 32 + e] = __uint_as_float(r[e]);
-        }
+        for (int e = 0; e < 32; ++e) v[c * 32 + e] = __uint_as_float(r[e]);
       }
-      tc_fence_before();
-      mbar_arrive(&bar->s_empty[sb]);
 
       float c_j = sl2, bias = 0.f;
       if constexpr (FP8) {
@@ -316,10 +349,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < BN; ++e)
           if (e >= valid) v[e] = -INFINITY;
       }
-      float mx = v[0];
+      float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
 #pragma unroll
-      for (int e = 1; e < BN; ++e) mx = fmaxf(mx, v[e]);
-      mx *= c_j;
+      for (int e = 4; e < BN - 4; e += 8) {
+        mx0 = max3(mx0, v[e + 0], v[e + 1]);
+        mx1 = max3(mx1, v[e + 2], v[e + 3]);
+        mx2 = max3(mx2, v[e + 4], v[e + 5]);
+        mx3 = max3(mx3, v[e + 6], v[e + 7]);
+      }
+      mx0 = max3(mx0, v[BN - 4], v[BN - 3]);
+      mx1 = max3(mx1, v[BN - 2], v[BN - 1]);
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_j;
       const float m_new = fmaxf(m_run, mx);
       float alpha = 1.f;
       const bool resc = (m_new - m_run) > kRescaleThreshold;
@@ -328,65 +368,63 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         m_run = m_new;
         l_run *= alpha;
       }
-      const float neg_m = bias - m_run;
-      float ls = 0.f;
-      uint32_t pk[C::P_COLS];
-      if constexpr (FP8) {
+      __syncwarp();
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        // O_t is stable here: PV_t(j-1) completed before S_t(j) was signalled.
 #pragma unroll
-        for (int c = 0; c < C::P_COLS; ++c) {
-          const float p0 = ex2_approx(fmaf(v[4 * c + 0], c_j, neg_m));
-          const float p1 = ex2_approx(fmaf(v[4 * c + 1], c_j, neg_m));
-          const float p2 = ex2_approx(fmaf(v[4 * c + 2], c_j, neg_m));
-          const float p3 = ex2_approx(fmaf(v[4 * c + 3], c_j, neg_m));
-          ls += (p0 + p1) + (p2 + p3);
-          pk[c] = pack_e4m3x4(p0, p1, p2, p3);
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(to + c * 32, r);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          tmem_st32(to + c * 32, r);
         }
-        ls *= ex2_approx(-bias);
+      }
+
+      const float neg_m = bias - m_run;
+      const float2 c2 = make_float2(c_j, c_j);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+      if constexpr (FP8) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float2 x0 = __ffma2_rn(make_float2(v[4 * c + 0], v[4 * c + 1]), c2, nm2);
+          const float2 x1 = __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), c2, nm2);
+          const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+          const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+          acc0 = __fadd2_rn(acc0, e0);
+          acc1 = __fadd2_rn(acc1, e1);
+          pk[c] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+        }
+        tmem_st32(ts, pk);
       } else {
 #pragma unroll
-        for (int c = 0; c < C::P_COLS; ++c) {
-          const float p0 = ex2_approx(fmaf(v[2 * c + 0], c_j, neg_m));
-          const float p1 = ex2_approx(fmaf(v[2 * c + 1], c_j, neg_m));
-          ls += p0 + p1;
-          pk[c] = KIND == 1 ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
-        }
-      }
-      l_run += ls;
-
-      if (j > 0) {
-        // P_{j-1} consumed and O final up to tile j-1 before P_j / rescale.
-        ok = warp_wait(&bar->o_done, (j - 1) & 1, ctl);
-        if (!ok) break;
-        __syncwarp();
-        tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          uint32_t r[32];
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            const uint32_t to = tmem + lane_base + kColO + c * 32;
-            tmem_ld32(to, r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            tmem_st32(to, r);
+          for (int c = 0; c < 32; c += 2) {
+            const int e = half * 64 + 2 * c;
+            const float2 x0 = __ffma2_rn(make_float2(v[e + 0], v[e + 1]), c2, nm2);
+            const float2 x1 = __ffma2_rn(make_float2(v[e + 2], v[e + 3]), c2, nm2);
+            const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+            const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+            acc0 = __fadd2_rn(acc0, e0);
+            acc1 = __fadd2_rn(acc1, e1);
+            pk[c] = KIND == 1 ? pack_bf16x2(e0.x, e0.y) : pack_f16x2(e0.x, e0.y);
+            pk[c + 1] = KIND == 1 ? pack_bf16x2(e1.x, e1.y) : pack_f16x2(e1.x, e1.y);
           }
+          tmem_st32(ts + half * 32, pk);
         }
       }
-      __syncwarp();
-      {
-        const uint32_t tp = tmem + lane_base + kColP;
-#pragma unroll
-        for (int c = 0; c < C::P_COLS / 32; ++c) {
-          uint32_t r[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) r[e] = pk[c * 32 + e];
-          tmem_st32(tp + c * 32, r);
-        }
-      }
+      float ls = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      if constexpr (FP8) ls *= ex2_approx(-bias);
+      l_run += ls;
       tc_fence_before();
-      mbar_arrive(&bar->p_full);
+      mbar_arrive(&bar->p_full[t]);
     }
 
-    if (ok) ok = warp_wait(&bar->o_done, (n_kv - 1) & 1, ctl);
+    if (ok) ok = warp_wait(&bar->o_final[t], 0, ctl);
     if (ok) {
       __syncwarp();
       tc_fence_after();
@@ -397,15 +435,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
         __syncwarp();
-        tmem_ld32(tmem + lane_base + kColO + c * 32, r);
+        tmem_ld32(to + c * 32, r);
         if (q_row < p.S) {
           uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(r[2 * e]) * out_scale,
-                                                      __uint_as_float(r[2 * e + 1]) * out_scale);
-            w[e] = *reinterpret_cast<uint32_t*>(&h2);
-          }
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * out_scale, __uint_as_float(r[2 * e + 1]) * out_scale);
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
@@ -433,7 +468,7 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMa
   auto kern = attn_fwd_kernel<D, KIND>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_tiles, p.B * p.H);
+  dim3 grid((p.n_tiles + NQ - 1) / NQ, p.B * p.H);
   kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
