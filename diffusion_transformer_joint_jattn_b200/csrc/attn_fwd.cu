@@ -330,12 +330,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncwarp();
       tc_fence_after();
       float v[BN];
+      {
+        uint32_t r[BN];
+        tmem_ld128(ts, r);
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(ts + c * 32, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[c * 32 + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(r[e]);
       }
 
       float c_j = sl2, bias = 0.f;
@@ -489,6 +488,8 @@ __global__ void selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
 }
 
 }  // namespace
+
+int fwd_kv_rows() { return BN; }
 
 cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {

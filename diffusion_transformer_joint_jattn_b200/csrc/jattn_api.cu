@@ -3,6 +3,7 @@
 // stream, and the per-device status word.
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -67,15 +68,15 @@ jattn_status check_shape(const jattn_shape* s) {
 int total_S(const jattn_shape* s) { return s->S_txt + s->S_img + s->S_ref; }
 int n_blocks(int S) { return (S + JATTN_BLOCK - 1) / JATTN_BLOCK; }
 
-// [BH][S][d] tensor map with (d-inner) boxes of box_inner elements x 128 rows.
-jattn_status make_map(CUtensorMap* m, const void* base, int BH, int S, int d, int elem_bytes) {
+// [BH][S][d] tensor map; boxes of (one swizzle span of d) x box_rows rows.
+jattn_status make_map(CUtensorMap* m, const void* base, int BH, int S, int d, int elem_bytes, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return JATTN_ERR_CUDA;
   const int row_bytes = d * elem_bytes;
   const int sw_bytes = row_bytes >= 128 ? 128 : 64;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(S), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * S};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(sw_bytes / elem_bytes), 128u, 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(sw_bytes / elem_bytes), static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const CUtensorMapSwizzle sw = sw_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -173,6 +174,10 @@ static jattn_status fwd_common(const jattn_shape* shape, const void* q, const vo
   p.lse = lse;
   p.status = status_ptr();
   p.timeout_ns = kDefaultTimeoutNs;
+  p.trace = nullptr;
+#ifdef JATTN_TRACE
+  if (const char* env = std::getenv("JATTN_TRACE_PTR")) p.trace = reinterpret_cast<long long*>(std::strtoull(env, nullptr, 0));
+#endif
   if (p.status == nullptr) return JATTN_ERR_CUDA;
   return JATTN_OK;
 }
@@ -185,9 +190,10 @@ jattn_status jattn_fwd_bf16(const jattn_shape* shape, jattn_dtype in_dtype, cons
   if (st != JATTN_OK) return st;
   CUtensorMap tq, tk, tv;
   const int BH = p.B * p.H;
-  if ((st = make_map(&tq, q, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
-  if ((st = make_map(&tk, k, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
-  if ((st = make_map(&tv, v, BH, p.S, shape->d, 2)) != JATTN_OK) return st;
+  const int kv_rows = jattn::fwd_kv_rows();
+  if ((st = make_map(&tq, q, BH, p.S, shape->d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
   return jattn::launch_fwd_f16(p, shape->d, in_dtype == JATTN_BF16, tq, tk, tv,
                                static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? JATTN_OK
@@ -203,9 +209,10 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
   p.scales = scales;
   CUtensorMap tq, tk, tv;
   const int BH = p.B * p.H;
-  if ((st = make_map(&tq, q8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
-  if ((st = make_map(&tk, k8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
-  if ((st = make_map(&tv, v8, BH, p.S, shape->d, 1)) != JATTN_OK) return st;
+  const int kv_rows = jattn::fwd_kv_rows();
+  if ((st = make_map(&tq, q8, BH, p.S, shape->d, 1, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k8, BH, p.S, shape->d, 1, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v8, BH, p.S, shape->d, 1, kv_rows)) != JATTN_OK) return st;
   return jattn::launch_fwd_fp8(p, shape->d, tq, tk, tv, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? JATTN_OK
              : JATTN_ERR_CUDA;
@@ -220,6 +227,7 @@ jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits) {
   if (cudaMemcpy(&w, ptr, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return JATTN_ERR_CUDA;
   if (clear && cudaMemset(ptr, 0, sizeof(uint32_t)) != cudaSuccess) return JATTN_ERR_CUDA;
   if (bits != nullptr) *bits = w;
+  if (w & JATTN_DEV_CHECK) return JATTN_ERR_INTERNAL;
   if (w & JATTN_DEV_TIMEOUT) return JATTN_ERR_TIMEOUT;
   if (w & JATTN_DEV_RANGE) return JATTN_ERR_RANGE;
   return JATTN_OK;
@@ -244,6 +252,7 @@ const char* jattn_status_string(jattn_status s) {
     case JATTN_ERR_CUDA: return "CUDA error";
     case JATTN_ERR_TIMEOUT: return "device wait timed out";
     case JATTN_ERR_RANGE: return "value out of 16-bit range (saturated)";
+    case JATTN_ERR_INTERNAL: return "kernel internal check failed";
   }
   return "unknown status";
 }

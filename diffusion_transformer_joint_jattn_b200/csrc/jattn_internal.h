@@ -36,6 +36,7 @@ struct FwdParams {
   const float* scales;          // fp8: [3][B][H][n_tiles]
   uint32_t* status;
   uint64_t timeout_ns;
+  long long* trace;             // development timing probe; always null in the library
 };
 
 // out_kind: 0 = fp16, 1 = bf16, 2 = e4m3
@@ -48,6 +49,9 @@ cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtens
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st);
 cudaError_t launch_fwd_fp8(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, cudaStream_t st);
+
+// Rows of the K / V tiles the forward kernels walk (the TMA box height).
+int fwd_kv_rows();
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 

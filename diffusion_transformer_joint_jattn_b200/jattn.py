@@ -24,8 +24,8 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libjattn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
-DEV_TIMEOUT, DEV_RANGE = 1, 2
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_ALIGNMENT, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_INTERNAL = range(8)
+DEV_TIMEOUT, DEV_RANGE, DEV_CHECK = 1, 2, 4
 BF16, FP16, E4M3 = 0, 1, 2
 BLOCK = 128
 

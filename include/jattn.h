@@ -53,12 +53,14 @@ typedef enum {
   JATTN_ERR_ALIGNMENT = 3,
   JATTN_ERR_CUDA = 4,
   JATTN_ERR_TIMEOUT = 5, /* a kernel gave up waiting; see jattn_device_status */
-  JATTN_ERR_RANGE = 6    /* a value exceeded the 16-bit output range (saturated) */
+  JATTN_ERR_RANGE = 6,   /* a value exceeded the 16-bit output range (saturated) */
+  JATTN_ERR_INTERNAL = 7 /* a kernel's internal consistency check failed */
 } jattn_status;
 
 /* Bits of the device status word. */
 #define JATTN_DEV_TIMEOUT 1u
 #define JATTN_DEV_RANGE 2u
+#define JATTN_DEV_CHECK 4u
 
 typedef enum { JATTN_BF16 = 0, JATTN_FP16 = 1, JATTN_E4M3 = 2 } jattn_dtype;
 
@@ -136,7 +138,8 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
 
 /*
  * Synchronise `stream`, read the current device's status word and return
- * JATTN_OK, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (timeout wins).  The raw
+ * JATTN_OK, JATTN_ERR_INTERNAL, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (in
+ * that order of precedence).  The raw
  * bits go to *bits if bits is non-NULL.  clear != 0 resets the word.
  */
 jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits);
