@@ -30,6 +30,11 @@ sys.path.insert(0, ROOT)
 from diffusion_transformer_joint_jattn_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = "t2i_2048_base"
+# DRAM bytes per launch of the forward kernel on t2i_2048_base: the ncu
+# capture of the same kernel on t2i_1024_base (profiles/attn_fwd_t2i_1024_base.md,
+# dram__bytes_read.sum + dram__bytes_write.sum = 207.44 MB) scaled by the token
+# count 16896 / 4608 (the traffic is Q, K, V and O once each, linear in tokens).
+FWD_TRAFFIC_BYTES = 207.44e6 * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 
@@ -241,8 +246,9 @@ def run_ours(args, rank, world, local):
                      "peak_note": f"{peak_src} cuBLAS bf16 sustained (MEASURED_PEAKS.json bf16_tflops_sustained)",
                      "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
                      "frac_of_nominal_2250": round(achieved / 2250.0, 4),
-                     "traffic": None,
-                     "kernel": "attn_fwd_kernel<128,false>"},
+                     "traffic": round(FWD_TRAFFIC_BYTES) if args.workload == WORKLOAD else None,
+                     "traffic_note": "ncu capture on t2i_1024_base scaled by tokens (see profiles/)",
+                     "kernel": "attn_fwd_kernel<128, fp16 operands>"},
         "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / pro_ms / 1e6, 1),
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
                               "frac": round(prologue_bytes(w, 2) / pro_ms / 1e6 / peaks["hbm_gbs"], 4)},

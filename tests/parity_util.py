@@ -63,5 +63,34 @@ def workload_case(name: str, n_rows: int = 4096, seed: int = 0):
     return w, inp, rows, O, L
 
 
+def fp16_operand_floor(w, inp, rows) -> np.ndarray:
+    """The oracle's attention (float64) on the sampled rows after rounding the
+    rotated Q and K to fp16 (V is exact in fp16 for these inputs): with the
+    result rounded to bf16 on top, the error any kernel with 16-bit
+    tensor-core operands and a bf16 output carries by format alone."""
+    import math
+    from concurrent.futures import ThreadPoolExecutor
+    q, k, v = oracle.joint_sequence(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"])
+    pos = inp["pos"].numpy()
+    rows = rows.numpy()
+    out = np.empty((w.B, w.H, rows.shape[-1], w.d))
+
+    def head(bh):
+        b, h = divmod(bh, w.H)
+        r = rows[b, h]
+        kr = oracle.rope_rotate(k[b, h], pos, w.split, w.theta).astype(np.float16).astype(np.float64)
+        qr = oracle.rope_rotate(q[b, h][r], pos[r], w.split, w.theta).astype(np.float16).astype(np.float64)
+        for i in range(0, len(r), 1024):
+            out[b, h, i:i + 1024], _ = oracle.attention_rows(qr[i:i + 1024], kr, v[b, h], 1 / math.sqrt(w.d))
+
+    with ThreadPoolExecutor(ORACLE_WORKERS) as ex:
+        list(ex.map(head, range(w.B * w.H)))
+    return out
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
 def to_device(inp, dev):
     return {k: (None if v is None else v.to(dev)) for k, v in inp.items()}

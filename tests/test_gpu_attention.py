@@ -4,8 +4,13 @@ C ABI.
 
 BF16 path (bf16 in, fp16 operands in the MMAs, bf16 out): rel-L2 <= 5e-3 and
 max-abs <= 2e-2 over the sampled rows (all rows for the small cases, 4096
-rows per (b, h) for the large workloads).  The pure-bf16-operand variant is
-checked against its own format floor (see the design notes).
+rows per (b, h) for the large workloads).  On the outlier workloads the
+max-abs bar lies below what 16-bit tensor-core operands can reach at all:
+the oracle itself, run on fp16-rounded rotated Q/K with a bf16 result,
+already shows max-abs 2.7e-2 .. 5e-2 there.  Those tests therefore assert
+max-abs within 1.25x of that measured floor (and 2e-2 where the floor is
+below it), plus the kernel's own deviation from the floored oracle.  The
+pure-bf16-operand variant is checked against its own format floor.
 """
 import numpy as np
 import pytest
@@ -14,8 +19,8 @@ import torch
 import oracle
 from diffusion_transformer_joint_jattn_b200 import jattn
 from diffusion_transformer_joint_jattn_b200 import workloads as W
-from parity_util import (BF16_MAX_ABS, BF16_REL_L2, gather_lse, gather_rows, max_abs, rel_l2, to_device,
-                         workload_case)
+from parity_util import (BF16_MAX_ABS, BF16_REL_L2, fp16_operand_floor, gather_lse, gather_rows, max_abs,
+                         rel_l2, round_bf16, to_device, workload_case)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,10 +86,18 @@ def test_workload_bf16_sampled_rows(cuda_device, name):
     w, inp, rows, O, L = workload_case(name)
     o, lse = _run_bf16(w, inp, cuda_device)
     got = gather_rows(o, rows)
+    floor = fp16_operand_floor(w, inp, rows)              # float64, fp16 Q/K operands
     r, m = rel_l2(got, O), max_abs(got, O)
-    print(f"{name}: rel-L2 {r:.3e} max-abs {m:.3e}")
-    assert r <= BF16_REL_L2 and m <= BF16_MAX_ABS
-    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=0, atol=5e-3)
+    rf, mf = rel_l2(round_bf16(floor), O), max_abs(round_bf16(floor), O)
+    r_kernel = rel_l2(got, floor)
+    print(f"{name}: rel-L2 {r:.3e} max-abs {m:.3e} | fp16-operand floor (bf16 out) rel-L2 {rf:.3e} "
+          f"max-abs {mf:.3e} | kernel vs fp16-operand oracle rel-L2 {r_kernel:.3e}")
+    assert r <= BF16_REL_L2
+    assert m <= max(BF16_MAX_ABS, 1.25 * mf)
+    assert r_kernel <= 2.5e-3
+    # LSE ~ the row's largest logit (up to ~40 here); fp16 rounding of the
+    # rotated Q/K makes its error relative (~7e-4), hence rtol.
+    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=2e-3, atol=5e-3)
     assert jattn.device_status()[0] == jattn.OK
 
 
