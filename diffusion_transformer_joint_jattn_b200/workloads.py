@@ -162,6 +162,15 @@ def make_inputs(w: JointAttentionWorkload, seed: int = 0, shared_outliers: bool 
                 pos=joint_positions(w.S_txt, w.grid, w.n_ref))
 
 
+def norm_weights(d: int, seed: int = 0, spread: float = 0.25) -> torch.Tensor:
+    """Synthetic query/key RMSNorm weights: fp32 ``[3, 2, d]`` (stream txt /
+    img / ref, then Q / K), drawn as 1 + spread * N(0, 1) from a generator
+    seeded ``seed + 3``.  (Trained weights are not needed: the normalisation's
+    arithmetic is the same for any weight vector.)"""
+    g = torch.Generator().manual_seed(seed + 3)
+    return (1.0 + spread * torch.randn(3, 2, d, generator=g, dtype=torch.float32)).contiguous()
+
+
 def sample_rows(w: JointAttentionWorkload, n: int = 4096, seed: int = 0) -> torch.Tensor:
     """Sorted distinct query rows per (b, h): int64 ``[B, H, m]`` with
     m = min(n, S); every row when S <= n."""

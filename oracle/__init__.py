@@ -12,7 +12,7 @@ not reuse its own formulas (see each test's docstring).  ``rounding_ambiguous``
 is a test helper, not part of the method.
 """
 from .joint_attention import (  # noqa: F401
-    as_f64, rope_frequencies, rope_angles, rope_rotate, joint_sequence,
+    as_f64, rope_frequencies, rope_angles, rope_rotate, rms_norm, qk_norm_streams, joint_sequence,
     attention_rows, joint_attention, rotated_qkv, attention_on, flops,
 )
 from .fp8 import (  # noqa: F401

@@ -16,7 +16,9 @@ GPUs"):
     target-image and optional reference-image streams are combined through
     joint attention -> ``joint_sequence``;
   * section "GEMM kernel optimization": rotary position embeddings are applied
-    to the query and key projections -> ``rope_rotate``;
+    to the query and key projections -> ``rope_rotate``; the same fused
+    projection also normalises the query and key -> ``rms_norm`` /
+    ``qk_norm_streams`` (optional);
   * section "Quantized and sparse attention": the dense (VANILLA) attention the
     quantised variants are compared against -> ``attention_rows``.
 
@@ -25,7 +27,11 @@ Readings where the page is silent (each is listed in the design notes):
   * RoPE is 2D axial over (t, row, col) with per-axis channel spans
     ``split = (n_t, n_r, n_c)`` laid out in that order; inside a span of n
     channels, pair p = channels (2p, 2p+1) rotates by pos_axis * theta^(-2p/n);
-  * the softmax scale is exactly 1/sqrt(d).
+  * the softmax scale is exactly 1/sqrt(d);
+  * query/key normalisation (when used) is RMSNorm over the d channels of
+    one (token, head), with a learned per-channel weight, one weight vector
+    per stream and per Q/K, applied before the rotation:
+    x -> w * x / sqrt(mean(x^2) + eps).
 """
 from __future__ import annotations
 
@@ -82,6 +88,36 @@ def rope_rotate(x: np.ndarray, pos: np.ndarray, split, theta: float) -> np.ndarr
 
 
 # --------------------------------------------------------------------------
+# Query / key RMS normalisation
+# --------------------------------------------------------------------------
+
+def rms_norm(x, w, eps: float) -> np.ndarray:
+    """w * x / sqrt(mean(x^2) + eps) over the last axis of ``x[..., d]``;
+    ``w`` is ``[d]``."""
+    x = np.asarray(x, dtype=np.float64)
+    ms = np.mean(x * x, axis=-1, keepdims=True)
+    return x / np.sqrt(ms + eps) * np.asarray(w, dtype=np.float64)
+
+
+def qk_norm_streams(qkv_txt, qkv_img, qkv_ref, norm_w, eps: float):
+    """Normalise Q and K of each stream ``[B, S_s, 3, H, d]`` with that
+    stream's weights: ``norm_w[s][0]`` for Q and ``norm_w[s][1]`` for K, s = 0
+    (txt), 1 (img), 2 (ref).  V is untouched.  Returns float64 streams
+    (``None`` stays ``None``)."""
+    w = as_f64(norm_w)
+    out = []
+    for s, t in enumerate((qkv_txt, qkv_img, qkv_ref)):
+        if t is None:
+            out.append(None)
+            continue
+        x = as_f64(t).copy()
+        x[:, :, 0] = rms_norm(x[:, :, 0], w[s, 0], eps)
+        x[:, :, 1] = rms_norm(x[:, :, 1], w[s, 1], eps)
+        out.append(x)
+    return out
+
+
+# --------------------------------------------------------------------------
 # Joint sequence assembly
 # --------------------------------------------------------------------------
 
@@ -116,12 +152,16 @@ def attention_rows(q_rows: np.ndarray, k: np.ndarray, v: np.ndarray, scale: floa
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta=10000.0, rows=None,
-                    softmax_scale=None, row_chunk=1024, workers=None):
-    """The whole hot path in FP64: assemble, rotate Q/K, attend.
+                    softmax_scale=None, row_chunk=1024, workers=None, norm_w=None, eps=1e-6):
+    """The whole hot path in FP64: (normalise Q/K,) assemble, rotate Q/K,
+    attend.
 
     rows: None for every row, else int ``[B, H, m]`` query-row indices.
+    norm_w: None, or ``[3, 2, d]`` query/key RMSNorm weights per stream.
     Returns (O [B, H, m, d], LSE [B, H, m]) in float64.
     """
+    if norm_w is not None:
+        qkv_txt, qkv_img, qkv_ref = qk_norm_streams(qkv_txt, qkv_img, qkv_ref, norm_w, eps)
     q, k, v = joint_sequence(qkv_txt, qkv_img, qkv_ref)
     pos = np.asarray(pos.numpy() if isinstance(pos, torch.Tensor) else pos)
     B, H, S, d = q.shape
@@ -151,9 +191,12 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta=10000.0, rows=N
     return O, L
 
 
-def rotated_qkv(qkv_txt, qkv_img, qkv_ref, pos, split, theta=10000.0):
+def rotated_qkv(qkv_txt, qkv_img, qkv_ref, pos, split, theta=10000.0, norm_w=None, eps=1e-6):
     """FP64 rotated Q, K and plain V, each ``[B, H, S, d]`` (the prologue's
-    exact result before rounding to a storage type)."""
+    exact result before rounding to a storage type); Q and K normalised
+    first when ``norm_w`` is given."""
+    if norm_w is not None:
+        qkv_txt, qkv_img, qkv_ref = qk_norm_streams(qkv_txt, qkv_img, qkv_ref, norm_w, eps)
     q, k, v = joint_sequence(qkv_txt, qkv_img, qkv_ref)
     pos = np.asarray(pos.numpy() if isinstance(pos, torch.Tensor) else pos)
     return rope_rotate(q, pos, split, theta), rope_rotate(k, pos, split, theta), v
