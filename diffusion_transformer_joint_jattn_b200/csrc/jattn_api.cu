@@ -89,13 +89,9 @@ float resolve_scale(float softmax_scale, int d) {
   return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
 }
 
-}  // namespace
-
-extern "C" {
-
-jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
-                            const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
-                            jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream) {
+jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img, const void* qkv_ref,
+                         const int32_t* pos, float theta, const int32_t split[3], const float* norm_w, float eps,
+                         jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream) {
   jattn_status st = check_shape(shape);
   if (st != JATTN_OK) return st;
   if (split == nullptr || pos == nullptr || q == nullptr || k == nullptr || v == nullptr) return JATTN_ERR_INVALID_ARG;
@@ -112,6 +108,7 @@ jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const
   if (out_dtype != JATTN_BF16 && out_dtype != JATTN_FP16 && out_dtype != JATTN_E4M3) return JATTN_ERR_UNSUPPORTED;
   if (out_dtype == JATTN_E4M3 && scales == nullptr) return JATTN_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(pos)) return JATTN_ERR_ALIGNMENT;
+  if (norm_w != nullptr && !aligned16(norm_w)) return JATTN_ERR_ALIGNMENT;
 
   jattn::RopeParams p{};
   for (int i = 0; i < 3; ++i) {
@@ -130,11 +127,33 @@ jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const
   p.dst[1] = k;
   p.dst[2] = v;
   p.scales = scales;
+  p.norm_w = norm_w;
+  p.eps = eps;
   p.status = status_ptr();
   if (p.status == nullptr) return JATTN_ERR_CUDA;
   const int kind = out_dtype == JATTN_FP16 ? 0 : (out_dtype == JATTN_BF16 ? 1 : 2);
   return jattn::launch_rope_qkv(p, kind, static_cast<cudaStream_t>(stream)) == cudaSuccess ? JATTN_OK
                                                                                           : JATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                            const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
+                            jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream) {
+  return rope_common(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, nullptr, 0.f, out_dtype, q, k, v, scales,
+                     stream);
+}
+
+jattn_status jattn_rope_qkv_norm(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                 const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
+                                 const float* norm_w, float eps, jattn_dtype out_dtype, void* q, void* k,
+                                 void* v, float* scales, void* stream) {
+  if (norm_w == nullptr || !(eps > 0.f) || !std::isfinite(eps)) return JATTN_ERR_INVALID_ARG;
+  return rope_common(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, norm_w, eps, out_dtype, q, k, v, scales,
+                     stream);
 }
 
 jattn_status jattn_quant_fp8(const jattn_shape* shape, jattn_dtype in_dtype, const void* x, void* x8,

@@ -18,6 +18,8 @@ struct RopeParams {
   int split[3];
   void* dst[3];                 // q, k, v [B, H, S, d]
   float* scales;                // e4m3 output: [3][B][H][nblk]
+  const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
+  float eps;                    // RMSNorm epsilon
   uint32_t* status;
 };
 

@@ -1,13 +1,17 @@
-// Prologue kernels: joint-sequence assembly + 2D axial RoPE on Q/K, with the
-// output either in a 16-bit type or quantised to e4m3 with one fp32 scale
-// per (batch, head, 128-token block); and the standalone block quantiser.
+// Prologue kernels: joint-sequence assembly + (optional query/key RMSNorm) +
+// 2D axial RoPE on Q/K, with the output either in a 16-bit type or quantised
+// to e4m3 with one fp32 scale per (batch, head, 128-token block); and the
+// standalone block quantiser.
 //
 // Method ("Speed Up Image Generation with FLUX 3 Image Klein on NVIDIA
 // Blackwell GPUs"): the text, target-image and reference-image streams are
 // joined for joint attention (section "FLUX 3 inference with TensorRT LLM
-// VisualGen"); rotary embeddings act on the query and key projections
-// (section "GEMM kernel optimization"); FP8 Q/K/V feed the quantised
-// attention (section "Quantized and sparse attention").
+// VisualGen"); rotary embeddings act on the query and key projections, which
+// the same fused projection also normalises (section "GEMM kernel
+// optimization"); FP8 Q/K/V feed the quantised attention (section "Quantized
+// and sparse attention").  The normalisation is taken as RMSNorm over the d
+// channels of one (token, head), w * x / sqrt(mean(x^2) + eps), with one
+// weight vector per stream and per Q/K, applied before the rotation.
 //
 // Design: HBM-bound streaming.  One CTA owns one 128-token block of one batch
 // entry and walks all 3*H (Q/K/V, head) tiles of it, so each (token, pair)
@@ -15,7 +19,9 @@
 // are 16-byte vectors, coalesced along d; the next tile's loads are issued
 // before the current tile is processed.  For e4m3 output the tile's amax is
 // reduced across the CTA before its codes are written, so every input byte is
-// read exactly once.
+// read exactly once.  The RMSNorm's sum of squares is a shuffle reduction over
+// the D/8 consecutive lanes that hold one row; its weights are staged in
+// shared memory once per CTA.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
@@ -82,15 +88,17 @@ __device__ __forceinline__ void pair_cos_sin(int32_t pos_axis, int i, int n, dou
   sincosf(static_cast<float>(r), &s, &c);
 }
 
-// OUT: output kind.  D: head dimension.
-template <int D, int OUT>
+// OUT: output kind.  D: head dimension.  NORM: RMSNorm Q and K first.
+template <int D, int OUT, bool NORM>
 __global__ void __launch_bounds__(D / 8 * kTok / kTokPerThread)
 rope_qkv_kernel(const RopeParams p) {
   constexpr int CG = D / 8;                           // 16-byte chunks per row
   constexpr int NT = CG * kTok / kTokPerThread;       // threads
   constexpr int ROWS_PER_PASS = kTok / kTokPerThread; // tokens covered by one pass
   constexpr int NWARP = NT / 32;
+  static_assert(CG <= 32 && 32 % CG == 0, "a row's lanes must sit inside one warp");
   __shared__ float red[2][NWARP];
+  __shared__ __align__(16) float wsm[NORM ? 6 * D : 4];   // [stream][q/k][D]
 
   const int tid = threadIdx.x;
   const int cg = tid % CG;
@@ -99,11 +107,16 @@ rope_qkv_kernel(const RopeParams p) {
   const int b = blockIdx.y;
   const int H = p.H, S = p.S;
   const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
+  if constexpr (NORM) {
+    for (int i = tid; i < 6 * D; i += NT) wsm[i] = p.norm_w[i];
+    __syncthreads();
+  }
 
   // Per-token source row base (element offset of [b, local, 0, 0, 0] in its
   // stream) and validity.
   const __nv_bfloat16* src[kTokPerThread];
   int tok[kTokPerThread];
+  int stream[kTokPerThread];
   bool valid[kTokPerThread];
   float cs[kTokPerThread][4], sn[kTokPerThread][4];
 #pragma unroll
@@ -113,8 +126,11 @@ rope_qkv_kernel(const RopeParams p) {
     valid[i] = t < S;
     const __nv_bfloat16* base = p.src[0];
     int len = p.S_part[0], local = t;
-    if (t >= p.S_part[0]) { base = p.src[1]; len = p.S_part[1]; local = t - p.S_part[0]; }
-    if (t >= p.S_part[0] + p.S_part[1]) { base = p.src[2]; len = p.S_part[2]; local = t - p.S_part[0] - p.S_part[1]; }
+    stream[i] = 0;
+    if (t >= p.S_part[0]) { base = p.src[1]; len = p.S_part[1]; local = t - p.S_part[0]; stream[i] = 1; }
+    if (t >= p.S_part[0] + p.S_part[1]) {
+      base = p.src[2]; len = p.S_part[2]; local = t - p.S_part[0] - p.S_part[1]; stream[i] = 2;
+    }
     src[i] = valid[i] ? base + (static_cast<size_t>(b) * len + local) * 3 * H * D + cg * 8 : nullptr;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -151,6 +167,21 @@ rope_qkv_kernel(const RopeParams p) {
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) {
       bf16x8_to_f32(cur[i], x[i]);
+      if (NORM && which < 2) {
+        // RMSNorm over the row's D channels: this thread holds 8 of them,
+        // the row's other chunks sit in the CG consecutive lanes around it.
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(x[i][e], x[i][e], ss);
+#pragma unroll
+        for (int o = CG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float r = __frsqrt_rn(fmaf(ss, 1.0f / D, p.eps));
+        const float4* wv = reinterpret_cast<const float4*>(wsm + (stream[i] * 2 + which) * D + cg * 8);
+        const float4 w0 = wv[0], w1 = wv[1];
+        const float wr[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[i][e] = x[i][e] * r * wr[e];
+      }
       if (which < 2) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -285,7 +316,8 @@ template <int D, int OUT>
 cudaError_t launch_rope_t(const RopeParams& p, cudaStream_t st) {
   constexpr int NT = D / 8 * kTok / kTokPerThread;
   dim3 grid(p.nblk, p.B);
-  rope_qkv_kernel<D, OUT><<<grid, NT, 0, st>>>(p);
+  if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true><<<grid, NT, 0, st>>>(p);
+  else rope_qkv_kernel<D, OUT, false><<<grid, NT, 0, st>>>(p);
   return cudaGetLastError();
 }
 

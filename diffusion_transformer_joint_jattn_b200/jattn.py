@@ -33,7 +33,7 @@ _DTYPE_CODE = {torch.bfloat16: BF16, torch.float16: FP16, torch.float8_e4m3fn: E
 _CODE_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, E4M3: torch.float8_e4m3fn}
 _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 
-SYMBOLS = ("jattn_rope_qkv", "jattn_quant_fp8", "jattn_fwd_bf16", "jattn_fwd_fp8",
+SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_bf16", "jattn_fwd_fp8",
            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -63,6 +63,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     vp, i32, f32 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float
     sp = ctypes.POINTER(Shape)
     lib.jattn_rope_qkv.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), i32, vp, vp, vp, vp, vp]
+    lib.jattn_rope_qkv_norm.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, i32, vp, vp, vp,
+                                        vp, vp]
     lib.jattn_quant_fp8.argtypes = [sp, i32, vp, vp, vp, vp]
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
@@ -115,8 +117,9 @@ def n_blocks(S: int) -> int:
 
 
 def rope_qkv(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float = 10000.0,
-             out_dtype="fp16", out=None, stream=None):
-    """Assemble the joint sequence and rotate Q/K.
+             out_dtype="fp16", out=None, stream=None, norm_w=None, eps: float = 1e-6):
+    """Assemble the joint sequence and rotate Q/K (after an RMSNorm of Q and K
+    when ``norm_w`` is given: fp32 CUDA [3, 2, d], stream x (Q, K)).
 
     qkv_*: bf16 CUDA tensors [B, S_part, 3, H, d] (None for an empty stream);
     pos: int32 CUDA [S, 3].  Returns (q, k, v, scales); scales is None unless
@@ -149,9 +152,17 @@ def rope_qkv(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float 
         q, k, v, scales = out
     sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
     shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
-    _check(lib.jattn_rope_qkv(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
-                              float(theta), sp, code, _ptr(q), _ptr(k), _ptr(v), _ptr(scales), _stream(stream)),
-           "jattn_rope_qkv")
+    if norm_w is None:
+        _check(lib.jattn_rope_qkv(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
+                                  float(theta), sp, code, _ptr(q), _ptr(k), _ptr(v), _ptr(scales),
+                                  _stream(stream)), "jattn_rope_qkv")
+    else:
+        _dev(norm_w, "norm_w", torch.float32)
+        if tuple(norm_w.shape) != (3, 2, d):
+            raise ValueError(f"norm_w must be [3, 2, {d}], got {tuple(norm_w.shape)}")
+        _check(lib.jattn_rope_qkv_norm(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref),
+                                       _ptr(pos), float(theta), sp, _ptr(norm_w), float(eps), code, _ptr(q),
+                                       _ptr(k), _ptr(v), _ptr(scales), _stream(stream)), "jattn_rope_qkv_norm")
     return q, k, v, scales
 
 
@@ -220,8 +231,10 @@ def selftest_wait_timeout(limit_ms: int = 50, stream=None):
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
-                    operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None):
-    """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8).
+                    operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None,
+                    norm_w=None, eps: float = 1e-6):
+    """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8),
+    with the query/key RMSNorm fused into rope_qkv when ``norm_w`` is given.
 
     Accepts CUDA tensors, or CPU tensors (then copied to the current device
     -- asynchronously when they are pinned -- and the output copied back,
@@ -233,11 +246,13 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
         dev = torch.device("cuda", torch.cuda.current_device())
         parts = [None if t is None else t.to(dev, non_blocking=True) for t in parts]
         pos = pos.to(dev, non_blocking=True)
+        if norm_w is not None:
+            norm_w = norm_w.to(dev, non_blocking=True)
     if path == "bf16":
-        q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream)
+        q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream, norm_w=norm_w, eps=eps)
         o, lse = fwd_bf16(q, k, v, want_lse=want_lse, stream=stream)
     elif path == "fp8":
-        q, k, v, sc = rope_qkv(*parts, pos, split, theta, "e4m3", stream=stream)
+        q, k, v, sc = rope_qkv(*parts, pos, split, theta, "e4m3", stream=stream, norm_w=norm_w, eps=eps)
         o, lse = fwd_fp8(q, k, v, sc, want_lse=want_lse, stream=stream)
     else:
         raise ValueError(f"unknown path {path!r}")

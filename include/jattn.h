@@ -100,6 +100,30 @@ jattn_status jattn_rope_qkv(const jattn_shape* shape, const void* qkv_txt, const
                             void* v, float* scales, void* stream);
 
 /*
+ * As jattn_rope_qkv, with query/key normalisation fused in front of the
+ * rotation ("Speed Up Image Generation with FLUX 3 Image Klein on NVIDIA
+ * Blackwell GPUs", section "GEMM kernel optimization": the fused QKV
+ * projection applies query/key normalisation and RoPE).  The page does not
+ * spell the normalisation out; it is taken as RMSNorm over the d channels of
+ * one (token, head), before the rotation:
+ *   x -> w[stream][Q or K][c] * x_c / sqrt(mean_c(x_c^2) + eps)
+ * computed in fp32 (sum of squares, then a correctly rounded 1/sqrt).
+ *   norm_w : device fp32 [3][2][d]: stream (0 = txt, 1 = img, 2 = ref), then
+ *            0 = Q, 1 = K.  Pass the same values twice to share weights
+ *            between streams.  Must not be NULL; 16-byte aligned.
+ *   eps    : > 0 and finite (1e-6 in the FLUX family); else
+ *            JATTN_ERR_INVALID_ARG.
+ * V is not normalised.  All other arguments, layouts and errors as
+ * jattn_rope_qkv; with out_dtype JATTN_E4M3 the block scales are those of
+ * the normalised, rotated values.
+ */
+jattn_status jattn_rope_qkv_norm(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                 const void* qkv_ref, const int32_t* pos, float theta,
+                                 const int32_t split[3], const float* norm_w, float eps,
+                                 jattn_dtype out_dtype, void* q, void* k, void* v, float* scales,
+                                 void* stream);
+
+/*
  * Per-block e4m3 quantisation of one laid-out 16-bit tensor.
  *   x      : in_dtype (JATTN_BF16 or JATTN_FP16) [B, H, S, d]
  *   x8     : e4m3 [B, H, S, d]

@@ -89,6 +89,22 @@ def test_rope_rejects_bad_arguments():
     assert f(shape(), A, None, None, A, 1e4, ok_split, 7, A, A, A, None, None) == jattn.ERR_UNSUPPORTED
 
 
+def test_rope_norm_rejects_bad_arguments():
+    """The RMSNorm variant: weights required, eps > 0 and finite, weights
+    16-byte aligned; the shared checks of jattn_rope_qkv still apply."""
+    lib = jattn.load()
+    ok_split = _split(16, 56, 56)
+    f = lib.jattn_rope_qkv_norm
+    args = lambda w, eps, sp=ok_split: (shape(), A, None, None, A, 1e4, sp, w, eps, jattn.FP16, A, A, A, None, None)
+    assert f(*args(None, 1e-6)) == jattn.ERR_INVALID_ARG
+    assert f(*args(A, 0.0)) == jattn.ERR_INVALID_ARG
+    assert f(*args(A, -1e-6)) == jattn.ERR_INVALID_ARG
+    assert f(*args(A, float("nan"))) == jattn.ERR_INVALID_ARG
+    assert f(*args(A, float("inf"))) == jattn.ERR_INVALID_ARG
+    assert f(*args(A + 4, 1e-6)) == jattn.ERR_ALIGNMENT
+    assert f(*args(A, 1e-6, _split(16, 56, 58))) == jattn.ERR_INVALID_ARG
+
+
 def test_quant_rejects_bad_arguments():
     lib = jattn.load()
     f = lib.jattn_quant_fp8

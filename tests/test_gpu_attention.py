@@ -101,6 +101,28 @@ def test_workload_bf16_sampled_rows(cuda_device, name):
     assert jattn.device_status()[0] == jattn.OK
 
 
+@pytest.mark.parametrize("case", SMALL[:4], ids=lambda c: f"B{c['B']}H{c['H']}d{c['d']}t{c['S_txt']}g{c['grid']}r{c['n_ref']}")
+def test_joint_attention_with_qk_norm(cuda_device, case):
+    """The whole path with the query/key RMSNorm fused into the prologue,
+    against the oracle's norm -> RoPE -> attention, every row."""
+    w = W.custom(**case)
+    inp = W.make_inputs(w, seed=21)
+    nw = W.norm_weights(w.d, 21)
+    d = to_device(inp, cuda_device)
+    q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "fp16",
+                                norm_w=nw.to(cuda_device))
+    o, lse = jattn.fwd_bf16(q, k, v, want_lse=True)
+    torch.cuda.synchronize()
+    O, L = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                                  norm_w=nw, eps=1e-6)
+    rows = torch.arange(w.S).expand(w.B, w.H, w.S)
+    got = gather_rows(o, rows)
+    assert rel_l2(got, O) <= BF16_REL_L2, rel_l2(got, O)
+    assert max_abs(got, O) <= BF16_MAX_ABS, max_abs(got, O)
+    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=0, atol=2e-3)
+    assert jattn.device_status()[0] == jattn.OK
+
+
 def test_host_buffers_end_to_end(cuda_device):
     """The public one-call API with host tensors: copies in, runs the path,
     copies out; same result as the device-tensor call."""

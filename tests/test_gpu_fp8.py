@@ -70,6 +70,26 @@ def test_fp8_kernel_against_dequantised_operands(cuda_device, case):
     assert jattn.device_status()[0] == jattn.OK
 
 
+def test_fp8_with_qk_norm(cuda_device):
+    """FP8 path with the fused query/key RMSNorm: against the oracle on the
+    dequantised (normalised, rotated) operands, and against the exact result."""
+    w = W.custom(B=2, H=2, d=128, S_txt=77, grid=9, n_ref=1)
+    inp = W.make_inputs(w, seed=23)
+    nw = W.norm_weights(128, 23)
+    d = to_device(inp, cuda_device)
+    q8, k8, v8, sc = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "e4m3",
+                                    norm_w=nw.to(cuda_device))
+    o, _ = jattn.fwd_fp8(q8, k8, v8, sc)
+    torch.cuda.synchronize()
+    dq, dk, dv = (_dequant(t, sc[i]) for i, t in enumerate((q8, k8, v8)))
+    O2, _ = oracle.attention_on(dq, dk, dv)
+    got = gather_rows(o, torch.arange(w.S).expand(w.B, w.H, w.S))
+    assert rel_l2(got, O2) <= KERNEL_VS_DEQUANT
+    O, _ = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                                  norm_w=nw, eps=1e-6)
+    assert rel_l2(got, O) <= 0.15
+
+
 @pytest.mark.parametrize("sv", [(1.0, 1.0), (1.0, 0.5), (0.5, 1.0), (1.0, 0.25), (2.0 ** -6, 1.0), (1.0, 0.125),
                                 (3.0, 0.75)])
 def test_fp8_value_scales_closed_form(cuda_device, sv):

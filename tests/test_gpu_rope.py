@@ -11,6 +11,11 @@ oracle, through the C ABI.
   (there an fp32-vs-fp64 last-bit difference may flip the code by one step);
   V codes and all scales of V bit-exact; Q/K scales within 1e-6.
 * Standalone quantiser: codes and scales bit-exact (its inputs are exact).
+* Query/key RMSNorm fused in front of the rotation (jattn_rope_qkv_norm): the
+  same bounds with the fp32 normalisation's error added (sum of 128 squares
+  and a correctly rounded 1/sqrt: a few 2^-24 relative, bounded here by
+  2^-18 of the pair's magnitude), and a 2^-17 ambiguity window for e4m3
+  codes.
 """
 import numpy as np
 import pytest
@@ -31,12 +36,13 @@ def _ulp16(y: np.ndarray, dtype) -> np.ndarray:
     return 2.0 ** (e - mant)
 
 
-def _check_rotated(got: torch.Tensor, ref: np.ndarray, dtype, name: str):
-    """got: 16-bit [..., d]; ref: float64 exact rotation [..., d]."""
+def _check_rotated(got: torch.Tensor, ref: np.ndarray, dtype, name: str, rel: float = 2.0 ** -20):
+    """got: 16-bit [..., d]; ref: float64 exact rotation [..., d]; rel: the
+    fp32 arithmetic's error bound relative to the pair's magnitude."""
     g = got.cpu().to(torch.float64).numpy()
     pair = np.sqrt(ref[..., 0::2] ** 2 + ref[..., 1::2] ** 2)
     pair = np.repeat(pair, 2, axis=-1)
-    bound = 0.5 * _ulp16(ref, dtype) * (1 + 2.0 ** -10) + 2.0 ** -20 * pair
+    bound = 0.5 * _ulp16(ref, dtype) * (1 + 2.0 ** -10) + rel * pair
     err = np.abs(g - ref)
     assert np.all(err <= bound), f"{name}: {np.sum(err > bound)} elements beyond the bound, worst {np.max(err / bound):.2f}x"
     exact = torch.from_numpy(ref).to(dtype).to(torch.float64).numpy()
@@ -96,6 +102,71 @@ def test_rope_e4m3_codes_and_scales(cuda_device, case):
         np.testing.assert_allclose(sc[i], scales, rtol=1e-6)
         inv = 1.0 / np.repeat(sc[i].astype(np.float64), 128, axis=-1)[..., :w.S, None]
         amb = oracle.rounding_ambiguous(x32.astype(np.float64) * inv)
+        mism = (got != codes) & ~amb
+        assert mism.sum() == 0, f"{mism.sum()} unexplained code mismatches"
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: f"B{c['B']}H{c['H']}d{c['d']}t{c['S_txt']}g{c['grid']}r{c['n_ref']}")
+@pytest.mark.parametrize("out", ["fp16", "bf16"])
+def test_rope_norm_16bit(cuda_device, case, out):
+    w = W.custom(**case)
+    inp = W.make_inputs(w, seed=13)
+    nw = W.norm_weights(w.d, 13)
+    dinp = to_device(inp, cuda_device)
+    q, k, v, _ = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                                out, norm_w=nw.to(cuda_device), eps=1e-6)
+    torch.cuda.synchronize()
+    qr, kr, vr = oracle.rotated_qkv(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                                    norm_w=nw, eps=1e-6)
+    dt = torch.float16 if out == "fp16" else torch.bfloat16
+    for name, got, ref in (("q", q, qr), ("k", k, kr)):
+        _check_rotated(got, ref, dt, name, rel=2.0 ** -18)
+    assert torch.equal(v.cpu(), torch.from_numpy(vr).to(dt))
+    assert jattn.device_status()[0] == jattn.OK
+
+
+def test_rope_norm_zero_rows_and_large_eps(cuda_device):
+    """An all-zero Q row stays zero (0 * 1/sqrt(eps)); a large eps shrinks the
+    result towards zero exactly as the formula says."""
+    w = W.custom(B=1, H=2, d=128, S_txt=3, grid=4, n_ref=0)
+    inp = W.make_inputs(w, 2)
+    inp["qkv_txt"][0, 1, 0, 1] = 0                       # token 1, Q, head 1
+    nw = W.norm_weights(128, 2)
+    dinp = to_device(inp, cuda_device)
+    for eps in (1e-6, 4.0):
+        q, k, _, _ = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], None, dinp["pos"], w.split, w.theta, "fp16",
+                                    norm_w=nw.to(cuda_device), eps=eps)
+        torch.cuda.synchronize()
+        assert torch.all(q[0, 1, 1].cpu() == 0)
+        qr, kr, _ = oracle.rotated_qkv(inp["qkv_txt"], inp["qkv_img"], None, inp["pos"], w.split, w.theta,
+                                       norm_w=nw, eps=eps)
+        _check_rotated(q, qr, torch.float16, "q", rel=2.0 ** -18)
+        _check_rotated(k, kr, torch.float16, "k", rel=2.0 ** -18)
+
+
+@pytest.mark.parametrize("case", CASES[:3], ids=lambda c: f"B{c['B']}H{c['H']}d{c['d']}S{c['S_txt']}")
+def test_rope_norm_e4m3(cuda_device, case):
+    w = W.custom(**case)
+    inp = W.make_inputs(w, seed=17)
+    nw = W.norm_weights(w.d, 17)
+    dinp = to_device(inp, cuda_device)
+    q8, k8, v8, sc = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split,
+                                    w.theta, "e4m3", norm_w=nw.to(cuda_device), eps=1e-6)
+    torch.cuda.synchronize()
+    qr, kr, vr = oracle.rotated_qkv(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                                    norm_w=nw, eps=1e-6)
+    sc = sc.cpu().numpy()
+    for i, (got, ref) in enumerate(((q8, qr), (k8, kr), (v8, vr))):
+        x32 = ref.astype(np.float32)
+        codes, scales = oracle.quantize_blocks(x32)
+        got = got.cpu().view(torch.uint8).numpy()
+        if i == 2:
+            np.testing.assert_array_equal(got, codes)
+            np.testing.assert_array_equal(sc[2], scales)
+            continue
+        np.testing.assert_allclose(sc[i], scales, rtol=2.0 ** -17)
+        inv = 1.0 / np.repeat(sc[i].astype(np.float64), 128, axis=-1)[..., :w.S, None]
+        amb = oracle.rounding_ambiguous(ref * inv, rel=2.0 ** -17)
         mism = (got != codes) & ~amb
         assert mism.sum() == 0, f"{mism.sum()} unexplained code mismatches"
 
