@@ -15,6 +15,9 @@ from .joint_attention import (  # noqa: F401
     as_f64, rope_frequencies, rope_angles, rope_rotate, rms_norm, qk_norm_streams, joint_sequence,
     attention_rows, joint_attention, rotated_qkv, attention_on, flops,
 )
+from .repair import (  # noqa: F401
+    repair_count, repair_scores, repair_select, repaired_attention_rows, repaired_attention,
+)
 from .fp8 import (  # noqa: F401
     E4M3_MAX, e4m3_decode, e4m3_encode, block_scales, quantize_blocks,
     dequantize_blocks, rounding_ambiguous,
