@@ -12,7 +12,9 @@ quantisation error and corrects them with a residual computed at higher
 precision.  The page names neither the error measure nor the form of the
 correction; the readings taken here (also listed in the design notes) are:
 
-  * per (batch, head), n = ceil(rho * S) tokens are repaired;
+  * per (batch, head), n = min(S, ceil(rho * S - 1e-3)) tokens are repaired
+    (the 1e-3 keeps a budget that lands a rounding error above an integer,
+    e.g. a float32 rho of 0.3 on 10 tokens, from taking one more token);
   * a token's quantisation error is measured by the e4m3 error bound of its
     key and value rows, which for a floating-point format is proportional to
     their magnitude: score_j = |k_j|^2 + |v_j|^2 (rotated, unquantised k);
@@ -30,8 +32,8 @@ import numpy as np
 
 
 def repair_count(S: int, rho: float) -> int:
-    """n = ceil(rho * S), capped at S (0 when rho == 0)."""
-    return min(S, int(math.ceil(rho * S - 1e-12))) if rho > 0 else 0
+    """n = ceil(rho * S - 1e-3), within [0, S] (0 when rho == 0)."""
+    return max(0, min(S, int(math.ceil(rho * S - 1e-3)))) if rho > 0 else 0
 
 
 def repair_scores(k_rot: np.ndarray, v: np.ndarray) -> np.ndarray:

@@ -29,9 +29,11 @@ def test_selection_by_hand():
 
 
 @pytest.mark.parametrize("S,rho,n", [(16896, 0.005, 85), (200, 0.005, 1), (1000, 0.005, 5), (7, 0.0, 0),
-                                     (7, 1.0, 7), (33280, 0.005, 167)])
+                                     (7, 1.0, 7), (33280, 0.005, 167), (10, 0.30000001192092896, 3),
+                                     (100, 1e-6, 0)])
 def test_repair_count(S, rho, n):
-    """n = ceil(rho * S): 84.48 -> 85, exactly 5.0 -> 5 (not 6)."""
+    """n = ceil(rho * S - 1e-3): 84.48 -> 85, exactly 5.0 -> 5 (not 6), the
+    float32 value of 0.3 on 10 tokens -> 3 (not 4)."""
     assert oracle.repair_count(S, rho) == n
 
 
