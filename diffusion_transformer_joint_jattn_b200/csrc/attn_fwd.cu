@@ -158,7 +158,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int qp = blockIdx.x;                           // pair of query tiles
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
-  const int n_kv = p.n_tiles;
+  const int n_kv = p.n_kv;
 
   if (threadIdx.x == 0) {
     mbar_init(&bar->q_full, 1);
@@ -325,6 +325,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const float p8_log2 = 8.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
 
     for (int j = 0; j < n_kv; ++j) {
+      // Keys left out of this pass (same for every row of the tile).
+      uint4 km = make_uint4(0u, 0u, 0u, 0u);
+      if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * n_kv + j);
       ok = warp_wait(&bar->s_full[t], j & 1, ctl);
       if (!ok) break;
       __syncwarp();
@@ -342,11 +345,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         c_j = sl2 * sq * sc_k[j];
         bias = __log2f(sc_v[j] / max_sv) + p8_log2;
       }
-      const int valid = p.S - j * BN;
+      const int valid = p.S_kv - j * BN;
       if (valid < BN) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)
           if (e >= valid) v[e] = -INFINITY;
+      }
+      if ((km.x | km.y | km.z | km.w) != 0u) {
+        const uint32_t kw[4] = {km.x, km.y, km.z, km.w};
+#pragma unroll
+        for (int e = 0; e < BN; ++e)
+          if ((kw[e >> 5] >> (e & 31)) & 1u) v[e] = -INFINITY;
       }
       float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
 #pragma unroll
@@ -380,7 +389,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
 
-      const float neg_m = bias - m_run;
+      // A row whose keys so far were all left out keeps m = -inf; its
+      // probabilities are exp2(-inf) = 0 either way.
+      const float neg_m = m_run == -INFINITY ? 0.f : bias - m_run;
       const float2 c2 = make_float2(c_j, c_j);
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
@@ -429,6 +440,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tc_fence_after();
       float out_scale = 1.f / l_run;
       if constexpr (FP8) out_scale *= max_sv * ex2_approx(-p8_log2);
+      float lse2 = m_run + __log2f(l_run);             // log2 units
+      // Merge with a partial result over other keys already in o:
+      // O = w_a O_a + w_b O_b with w = 2^(LSE_part - LSE), LSE = log2(2^a + 2^b).
+      float w_prev = 0.f;
+      if (p.lse_prev != nullptr && q_row < p.S) {
+        const float la = p.lse_prev[static_cast<size_t>(bh) * p.S + q_row] * 1.4426950408889634f;
+        if (la != -INFINITY) {
+          const float mx = fmaxf(la, lse2);
+          const float tot = mx + __log2f(ex2_approx(la - mx) + ex2_approx(lse2 - mx));
+          w_prev = ex2_approx(la - tot);
+          out_scale *= ex2_approx(lse2 - tot);
+          lse2 = tot;
+        }
+      }
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.S + q_row) * p.H + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
@@ -436,17 +461,34 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         __syncwarp();
         tmem_ld32(to + c * 32, r);
         if (q_row < p.S) {
+          float prev[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) prev[e] = 0.f;
+          if (w_prev != 0.f) {
+            const uint4* src = reinterpret_cast<const uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint4 u = src[e];
+              const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int f = 0; f < 4; ++f) {
+                prev[8 * e + 2 * f] = __uint_as_float(uw[f] << 16) * w_prev;
+                prev[8 * e + 2 * f + 1] = __uint_as_float(uw[f] & 0xFFFF0000u) * w_prev;
+              }
+            }
+          }
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * out_scale, __uint_as_float(r[2 * e + 1]) * out_scale);
+            w[e] = pack_bf16x2(fmaf(__uint_as_float(r[2 * e]), out_scale, prev[2 * e]),
+                               fmaf(__uint_as_float(r[2 * e + 1]), out_scale, prev[2 * e + 1]));
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
       if (p.lse != nullptr && q_row < p.S)
-        p.lse[static_cast<size_t>(bh) * p.S + q_row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        p.lse[static_cast<size_t>(bh) * p.S + q_row] = lse2 * 0.69314718055994531f;
     }
   }
 

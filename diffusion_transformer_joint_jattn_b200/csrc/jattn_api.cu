@@ -91,7 +91,8 @@ float resolve_scale(float softmax_scale, int d) {
 
 jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img, const void* qkv_ref,
                          const int32_t* pos, float theta, const int32_t split[3], const float* norm_w, float eps,
-                         jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream) {
+                         jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream,
+                         void* q16 = nullptr, float* score = nullptr) {
   jattn_status st = check_shape(shape);
   if (st != JATTN_OK) return st;
   if (split == nullptr || pos == nullptr || q == nullptr || k == nullptr || v == nullptr) return JATTN_ERR_INVALID_ARG;
@@ -129,11 +130,48 @@ jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const vo
   p.scales = scales;
   p.norm_w = norm_w;
   p.eps = eps;
+  p.q16 = q16;
+  p.score = score;
   p.status = status_ptr();
   if (p.status == nullptr) return JATTN_ERR_CUDA;
   const int kind = out_dtype == JATTN_FP16 ? 0 : (out_dtype == JATTN_BF16 ? 1 : 2);
   return jattn::launch_rope_qkv(p, kind, static_cast<cudaStream_t>(stream)) == cudaSuccess ? JATTN_OK
                                                                                           : JATTN_ERR_CUDA;
+}
+
+int repair_n(const jattn_shape* shape, float rho) {
+  const int S = total_S(shape);
+  if (!(rho > 0.f)) return 0;
+  const double x = std::ceil(static_cast<double>(rho) * S - 1e-3);
+  return x <= 0.0 ? 0 : (x >= S ? S : static_cast<int>(x));
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace segments, each 256-byte aligned, in this order.
+struct RepairLayout {
+  size_t q8, k8, v8, scales, q16, score, idx, kmask, kr, vr, lse, total;
+};
+
+RepairLayout repair_layout(const jattn_shape* shape, int n) {
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const size_t S = total_S(shape), d = shape->d, nb = n_blocks(static_cast<int>(S));
+  RepairLayout L{};
+  size_t off = 0;
+  auto seg = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+  L.q8 = seg(BH * S * d);
+  L.k8 = seg(BH * S * d);
+  L.v8 = seg(BH * S * d);
+  L.scales = seg(3 * BH * nb * 4);
+  L.q16 = seg(BH * S * d * 2);
+  L.score = seg(BH * S * 4);
+  L.idx = seg(BH * n * 4);
+  L.kmask = seg(BH * nb * 16);
+  L.kr = seg(BH * n * d * 2);
+  L.vr = seg(BH * n * d * 2);
+  L.lse = seg(BH * S * 4);
+  L.total = off;
+  return L;
 }
 
 }  // namespace
@@ -188,6 +226,10 @@ static jattn_status fwd_common(const jattn_shape* shape, const void* q, const vo
   p.H = shape->H;
   p.S = total_S(shape);
   p.n_tiles = n_blocks(p.S);
+  p.S_kv = p.S;
+  p.n_kv = p.n_tiles;
+  p.kmask = nullptr;
+  p.lse_prev = nullptr;
   p.scale_log2 = resolve_scale(softmax_scale, shape->d) * 1.4426950408889634f;
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
@@ -235,6 +277,99 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
   return jattn::launch_fwd_fp8(p, shape->d, tq, tk, tv, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? JATTN_OK
              : JATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- FP8 with token repair
+
+int32_t jattn_repair_count(const jattn_shape* shape, float rho) {
+  if (check_shape(shape) != JATTN_OK || !(rho >= 0.f && rho <= 1.f)) return -1;
+  return repair_n(shape, rho);
+}
+
+size_t jattn_fwd_fp8_repair_workspace(const jattn_shape* shape, float rho) {
+  if (check_shape(shape) != JATTN_OK || !(rho >= 0.f && rho <= 1.f)) return 0;
+  return repair_layout(shape, repair_n(shape, rho)).total;
+}
+
+jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                  const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
+                                  const float* norm_w, float eps, float rho, void* workspace,
+                                  size_t workspace_bytes, void* o, float* lse, int32_t* repaired,
+                                  float softmax_scale, void* stream) {
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  if (!(rho >= 0.f && rho <= 1.f)) return JATTN_ERR_INVALID_ARG;
+  if (norm_w != nullptr && (!(eps > 0.f) || !std::isfinite(eps))) return JATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || o == nullptr) return JATTN_ERR_INVALID_ARG;
+  const int n = repair_n(shape, rho);
+  const RepairLayout L = repair_layout(shape, n);
+  if (workspace_bytes < L.total) return JATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return JATTN_ERR_ALIGNMENT;
+  if (repaired != nullptr && (reinterpret_cast<uintptr_t>(repaired) & 3u)) return JATTN_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const int BH = shape->B * shape->H, S = total_S(shape), d = shape->d;
+  float* scales = reinterpret_cast<float*>(ws + L.scales);
+  float* score = reinterpret_cast<float*>(ws + L.score);
+  int32_t* idx = repaired != nullptr ? repaired : reinterpret_cast<int32_t*>(ws + L.idx);
+  uint32_t* kmask = reinterpret_cast<uint32_t*>(ws + L.kmask);
+  float* lse_a = lse != nullptr ? lse : reinterpret_cast<float*>(ws + L.lse);
+
+  // 1. Prologue: e4m3 Q/K/V + scales, and (with repairs) fp16 Q and the scores.
+  st = rope_common(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, norm_w, eps, JATTN_E4M3, ws + L.q8,
+                   ws + L.k8, ws + L.v8, scales, stream, n > 0 ? ws + L.q16 : nullptr, n > 0 ? score : nullptr);
+  if (st != JATTN_OK) return st;
+  // 2. Selection and 3. exact keys / values of the selected tokens.
+  if (n > 0) {
+    if (jattn::launch_repair_select(score, BH, S, n, n_blocks(S), idx, kmask, cs) != cudaSuccess)
+      return JATTN_ERR_CUDA;
+    jattn::GatherParams g{};
+    const void* parts[3] = {qkv_txt, qkv_img, qkv_ref};
+    const int lens[3] = {shape->S_txt, shape->S_img, shape->S_ref};
+    for (int i = 0; i < 3; ++i) {
+      g.src[i] = static_cast<const __nv_bfloat16*>(parts[i]);
+      g.S_part[i] = lens[i];
+      g.split[i] = split[i];
+    }
+    g.B = shape->B;
+    g.H = shape->H;
+    g.S = S;
+    g.d = d;
+    g.n = n;
+    g.pos = pos;
+    g.theta = static_cast<double>(theta);
+    g.norm_w = norm_w;
+    g.eps = eps;
+    g.idx = idx;
+    g.k_out = ws + L.kr;
+    g.v_out = ws + L.vr;
+    g.status = status_ptr();
+    if (jattn::launch_repair_gather(g, cs) != cudaSuccess) return JATTN_ERR_CUDA;
+  }
+  // 4. FP8 pass over the other keys.
+  jattn::FwdParams p{};
+  if ((st = fwd_common(shape, ws + L.q8, ws + L.k8, ws + L.v8, o, lse_a, softmax_scale, p)) != JATTN_OK) return st;
+  p.scales = scales;
+  p.kmask = n > 0 ? kmask : nullptr;
+  CUtensorMap tq, tk, tv;
+  const int kv_rows = jattn::fwd_kv_rows();
+  if ((st = make_map(&tq, ws + L.q8, BH, S, d, 1, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, ws + L.k8, BH, S, d, 1, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, ws + L.v8, BH, S, d, 1, kv_rows)) != JATTN_OK) return st;
+  if (jattn::launch_fwd_fp8(p, d, tq, tk, tv, cs) != cudaSuccess) return JATTN_ERR_CUDA;
+  if (n == 0) return JATTN_OK;
+  // 5. 16-bit pass over the repaired keys, merged into o (and lse).
+  jattn::FwdParams r = p;
+  r.scales = nullptr;
+  r.kmask = nullptr;
+  r.S_kv = n;
+  r.n_kv = n_blocks(n);
+  r.lse_prev = lse_a;
+  r.lse = lse;
+  if ((st = make_map(&tq, ws + L.q16, BH, S, d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, ws + L.kr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, ws + L.vr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
+  return jattn::launch_fwd_f16(r, d, false, tq, tk, tv, cs) == cudaSuccess ? JATTN_OK : JATTN_ERR_CUDA;
 }
 
 jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits) {

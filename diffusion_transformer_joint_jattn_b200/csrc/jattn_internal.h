@@ -20,8 +20,32 @@ struct RopeParams {
   float* scales;                // e4m3 output: [3][B][H][nblk]
   const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
   float eps;                    // RMSNorm epsilon
+  void* q16;                    // e4m3 output with token repair: also fp16 Q [B, H, S, d], else null
+  float* score;                 // with token repair: |k|^2 + |v|^2 per token [B, H, S], else null
   uint32_t* status;
 };
+
+// Exact (16-bit) keys and values of the repaired tokens.
+struct GatherParams {
+  const __nv_bfloat16* src[3];  // txt, img, ref streams [B, S_part, 3, H, d]
+  int S_part[3];
+  int B, H, S, d, n;            // n repaired tokens per (b, h)
+  const int32_t* pos;           // [S, 3]
+  double theta;
+  int split[3];
+  const float* norm_w;          // as RopeParams
+  float eps;
+  const int32_t* idx;           // [B*H][n] token indices
+  void* k_out;                  // fp16 [B*H][n][d], rotated (and normalised) keys
+  void* v_out;                  // fp16 [B*H][n][d]
+  uint32_t* status;
+};
+
+cudaError_t launch_repair_gather(const GatherParams& p, cudaStream_t st);
+// Per (b, h): the n largest scores (ties to the lower index) -> idx [B*H][n]
+// in index order, and the key mask [B*H][n_kv][4] words with their bits set.
+cudaError_t launch_repair_select(const float* score, int BH, int S, int n, int n_kv, int32_t* idx,
+                                 uint32_t* kmask, cudaStream_t st);
 
 struct QuantParams {
   const void* x;                // [BH, S, d] 16-bit
@@ -31,11 +55,15 @@ struct QuantParams {
 };
 
 struct FwdParams {
-  int B, H, S, n_tiles;         // n_tiles = ceil(S / 128)
+  int B, H, S, n_tiles;         // queries: S rows, n_tiles = ceil(S / 128)
+  int S_kv, n_kv;               // keys: S_kv rows (= S except for a residual pass), n_kv = ceil(S_kv / 128)
   float scale_log2;             // softmax_scale * log2(e)
   __nv_bfloat16* o;             // [B, S, H, d]
   float* lse;                   // [B, H, S] or null
   const float* scales;          // fp8: [3][B][H][n_tiles]
+  const uint32_t* kmask;        // null, or [B*H][n_kv][4] words: bit set = key left out of this pass
+  const float* lse_prev;        // null, or [B, H, S]: o already holds a partial result with this
+                                // LSE over other keys; the pass merges its own into o (and lse)
   uint32_t* status;
   uint64_t timeout_ns;
   long long* trace;             // development timing probe; always null in the library

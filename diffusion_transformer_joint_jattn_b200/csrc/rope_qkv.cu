@@ -89,7 +89,9 @@ __device__ __forceinline__ void pair_cos_sin(int32_t pos_axis, int i, int n, dou
 }
 
 // OUT: output kind.  D: head dimension.  NORM: RMSNorm Q and K first.
-template <int D, int OUT, bool NORM>
+// REPAIR (e4m3 output only): also write fp16 Q and the per-token repair score
+// |k|^2 + |v|^2 of the values that are quantised.
+template <int D, int OUT, bool NORM, bool REPAIR>
 __global__ void __launch_bounds__(D / 8 * kTok / kTokPerThread)
 rope_qkv_kernel(const RopeParams p) {
   constexpr int CG = D / 8;                           // 16-byte chunks per row
@@ -192,6 +194,42 @@ rope_qkv_kernel(const RopeParams p) {
       }
     }
     const size_t row0 = (static_cast<size_t>(b) * H + h) * S;
+
+    if constexpr (REPAIR) {
+      if (which == 0) {
+        uint16_t* q16 = static_cast<uint16_t*>(p.q16);
+#pragma unroll
+        for (int i = 0; i < kTokPerThread; ++i) {
+          if (!valid[i]) continue;
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            y[e] = x[i][e];
+            if (fabsf(y[e]) > 65504.f) {
+              range_hit = true;
+              y[e] = copysignf(65504.f, y[e]);
+            }
+          }
+          *reinterpret_cast<uint4*>(q16 + (row0 + tok[i]) * D + cg * 8) =
+              make_uint4(pack_f16(y[0], y[1]), pack_f16(y[2], y[3]), pack_f16(y[4], y[5]), pack_f16(y[6], y[7]));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kTokPerThread; ++i) {
+          float ss = 0.f;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(x[i][e], x[i][e], ss);
+#pragma unroll
+          for (int o = CG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+          if (cg == 0 && valid[i]) {
+            // K comes before V in the item order and the same lane owns the
+            // token in both, so the V pass reads back its own K term.
+            float* sc = p.score + row0 + tok[i];
+            *sc = which == 1 ? ss : *sc + ss;
+          }
+        }
+      }
+    }
 
     if constexpr (OUT == kOutE4M3) {
       float am = 0.f;
@@ -312,12 +350,96 @@ quant_fp8_kernel(const QuantParams p) {
   if (tid == 0) p.scales[bh * p.nblk + blk] = scale;
 }
 
+// Exact keys and values of the repaired tokens: one warp per (token, b, h);
+// the key row is (normalised and) rotated with the prologue's arithmetic and
+// both rows are stored as fp16.
+template <int D>
+__global__ void __launch_bounds__(256) repair_gather_kernel(const GatherParams p) {
+  constexpr int CPL = D / 32;                        // channels per lane (4 or 2)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r = blockIdx.x * 8 + warp;
+  const int bh = blockIdx.y;
+  if (r >= p.n) return;
+  const int b = bh / p.H, h = bh % p.H;
+  const int t = p.idx[static_cast<size_t>(bh) * p.n + r];
+  if (t < 0 || t >= p.S) {                           // not produced by the selection: report, write nothing
+    if (lane == 0) atomicOr(p.status, JATTN_DEV_CHECK);
+    return;
+  }
+  int stream = 0, local = t;
+  if (t >= p.S_part[0]) { stream = 1; local = t - p.S_part[0]; }
+  if (t >= p.S_part[0] + p.S_part[1]) { stream = 2; local = t - p.S_part[0] - p.S_part[1]; }
+  const __nv_bfloat16* row = p.src[stream] + (static_cast<size_t>(b) * p.S_part[stream] + local) * 3 * p.H * D;
+  const int c0 = lane * CPL;
+  float k[CPL], v[CPL];
+  {
+    const uint16_t* kr = reinterpret_cast<const uint16_t*>(row + (1 * p.H + h) * D + c0);
+    const uint16_t* vr = reinterpret_cast<const uint16_t*>(row + (2 * p.H + h) * D + c0);
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) {
+      k[e] = __uint_as_float(static_cast<uint32_t>(kr[e]) << 16);
+      v[e] = __uint_as_float(static_cast<uint32_t>(vr[e]) << 16);
+    }
+  }
+  if (p.norm_w != nullptr) {
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) ss = fmaf(k[e], k[e], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float rr = __frsqrt_rn(fmaf(ss, 1.0f / D, p.eps));
+    const float* w = p.norm_w + (stream * 2 + 1) * D + c0;
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) k[e] = k[e] * rr * w[e];
+  }
+  const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
+#pragma unroll
+  for (int j = 0; j < CPL / 2; ++j) {
+    int axis, ii, n;
+    pair_axis(c0 / 2 + j, n0, n1, n2, axis, ii, n);
+    float cs, sn;
+    pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs, sn);
+    const float a = k[2 * j], bb = k[2 * j + 1];
+    k[2 * j] = a * cs - bb * sn;
+    k[2 * j + 1] = a * sn + bb * cs;
+  }
+  bool range_hit = false;
+  uint32_t kw[CPL / 2], vw[CPL / 2];
+#pragma unroll
+  for (int e = 0; e < CPL; ++e) {
+    if (fabsf(k[e]) > 65504.f) { range_hit = true; k[e] = copysignf(65504.f, k[e]); }
+    if (fabsf(v[e]) > 65504.f) { range_hit = true; v[e] = copysignf(65504.f, v[e]); }
+  }
+#pragma unroll
+  for (int j = 0; j < CPL / 2; ++j) {
+    kw[j] = pack_f16(k[2 * j], k[2 * j + 1]);
+    vw[j] = pack_f16(v[2 * j], v[2 * j + 1]);
+  }
+  const size_t off = (static_cast<size_t>(bh) * p.n + r) * D + c0;
+  uint16_t* ko = static_cast<uint16_t*>(p.k_out) + off;
+  uint16_t* vo = static_cast<uint16_t*>(p.v_out) + off;
+  if constexpr (CPL == 4) {
+    *reinterpret_cast<uint2*>(ko) = make_uint2(kw[0], kw[1]);
+    *reinterpret_cast<uint2*>(vo) = make_uint2(vw[0], vw[1]);
+  } else {
+    *reinterpret_cast<uint32_t*>(ko) = kw[0];
+    *reinterpret_cast<uint32_t*>(vo) = vw[0];
+  }
+  if (range_hit) atomicOr(p.status, JATTN_DEV_RANGE);
+}
+
 template <int D, int OUT>
 cudaError_t launch_rope_t(const RopeParams& p, cudaStream_t st) {
   constexpr int NT = D / 8 * kTok / kTokPerThread;
   dim3 grid(p.nblk, p.B);
-  if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true><<<grid, NT, 0, st>>>(p);
-  else rope_qkv_kernel<D, OUT, false><<<grid, NT, 0, st>>>(p);
+  const bool repair = OUT == kOutE4M3 && p.score != nullptr;
+  if (repair) {
+    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, OUT == kOutE4M3><<<grid, NT, 0, st>>>(p);
+    else rope_qkv_kernel<D, OUT, false, OUT == kOutE4M3><<<grid, NT, 0, st>>>(p);
+  } else {
+    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, false><<<grid, NT, 0, st>>>(p);
+    else rope_qkv_kernel<D, OUT, false, false><<<grid, NT, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -340,6 +462,14 @@ cudaError_t launch_rope_qkv(const RopeParams& p, int out_kind, cudaStream_t st) 
   if (out_kind == 0) return launch_rope_t<64, kOutF16>(p, st);
   if (out_kind == 1) return launch_rope_t<64, kOutBF16>(p, st);
   return launch_rope_t<64, kOutE4M3>(p, st);
+}
+
+cudaError_t launch_repair_gather(const GatherParams& p, cudaStream_t st) {
+  if (p.n <= 0) return cudaSuccess;
+  dim3 grid((p.n + 7) / 8, p.B * p.H);
+  if (p.d == 128) repair_gather_kernel<128><<<grid, 256, 0, st>>>(p);
+  else repair_gather_kernel<64><<<grid, 256, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_fp8(const QuantParams& p, bool in_bf16, cudaStream_t st) {

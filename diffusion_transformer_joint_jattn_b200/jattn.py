@@ -33,7 +33,8 @@ _DTYPE_CODE = {torch.bfloat16: BF16, torch.float16: FP16, torch.float8_e4m3fn: E
 _CODE_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, E4M3: torch.float8_e4m3fn}
 _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 
-SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_bf16", "jattn_fwd_fp8",
+SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_fp8_repair",
+           "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_bf16", "jattn_fwd_fp8",
            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -66,6 +67,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jattn_rope_qkv_norm.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, i32, vp, vp, vp,
                                         vp, vp]
     lib.jattn_quant_fp8.argtypes = [sp, i32, vp, vp, vp, vp]
+    lib.jattn_fwd_fp8_repair.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, f32, vp,
+                                         ctypes.c_size_t, vp, vp, vp, f32, vp]
+    lib.jattn_fwd_fp8_repair_workspace.argtypes = [sp, f32]
+    lib.jattn_repair_count.argtypes = [sp, f32]
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -76,6 +81,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in SYMBOLS:
         if name not in ("jattn_status_string", "jattn_version"):
             getattr(lib, name).restype = i32
+    lib.jattn_fwd_fp8_repair_workspace.restype = ctypes.c_size_t
     _lib = lib
     return lib
 
@@ -228,6 +234,69 @@ def device_status(clear: bool = True, stream=None):
 
 def selftest_wait_timeout(limit_ms: int = 50, stream=None):
     _check(load().jattn_selftest_wait_timeout(int(limit_ms), _stream(stream)), "jattn_selftest_wait_timeout")
+
+
+def repair_count(B: int, H: int, S_txt: int, S_img: int, S_ref: int, d: int, rho: float) -> int:
+    """Tokens repaired per (b, h) for budget rho (jattn_repair_count)."""
+    n = load().jattn_repair_count(ctypes.byref(make_shape(B, H, S_txt, S_img, S_ref, d)), float(rho))
+    if n < 0:
+        raise ValueError("invalid shape or rho")
+    return n
+
+
+def repair_workspace_bytes(B: int, H: int, S_txt: int, S_img: int, S_ref: int, d: int, rho: float) -> int:
+    return load().jattn_fwd_fp8_repair_workspace(ctypes.byref(make_shape(B, H, S_txt, S_img, S_ref, d)),
+                                                 float(rho))
+
+
+def fwd_fp8_repair(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float = 10000.0,
+                   rho: float = 0.005, norm_w=None, eps: float = 1e-6, want_lse: bool = False,
+                   want_repaired: bool = False, softmax_scale: float = 0.0, workspace=None, o=None, lse=None,
+                   stream=None):
+    """The FP8 path with token repair in one call (jattn_fwd_fp8_repair).
+
+    Returns o bf16 [B, S, H, d], plus lse fp32 [B, H, S] and / or the
+    repaired token indices int32 [B, H, n] when asked for.  ``workspace``: a
+    uint8 CUDA tensor of at least repair_workspace_bytes(...) bytes (allocated
+    here when None)."""
+    lib = load()
+    parts = [qkv_txt, qkv_img, qkv_ref]
+    ref = next(t for t in parts if t is not None)
+    B, _, _, H, d = ref.shape
+    lens = []
+    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
+        if t is None:
+            lens.append(0)
+            continue
+        _dev(t, name, torch.bfloat16)
+        lens.append(t.shape[1])
+    S = sum(lens)
+    _dev(pos, "pos", torch.int32)
+    dev = ref.device
+    n = repair_count(B, H, *lens, d, rho)
+    need = repair_workspace_bytes(B, H, *lens, d, rho)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if o is None:
+        o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
+    if want_lse and lse is None:
+        lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    rep = torch.empty(B, H, n, dtype=torch.int32, device=dev) if want_repaired else None
+    if norm_w is not None:
+        _dev(norm_w, "norm_w", torch.float32)
+    sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
+    shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
+    _check(lib.jattn_fwd_fp8_repair(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
+                                    float(theta), sp, _ptr(norm_w), float(eps), float(rho), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _ptr(o), _ptr(lse),
+                                    _ptr(rep if rep is not None and rep.numel() else None), float(softmax_scale),
+                                    _stream(stream)), "jattn_fwd_fp8_repair")
+    out = [o]
+    if want_lse:
+        out.append(lse)
+    if want_repaired:
+        out.append(rep)
+    return out[0] if len(out) == 1 else tuple(out)
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",

@@ -161,6 +161,49 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
                            float softmax_scale, void* stream);
 
 /*
+ * FP8 attention with token repair ("Speed Up Image Generation with FLUX 3
+ * Image Klein on NVIDIA Blackwell GPUs", section "Quantized and sparse
+ * attention": a repair budget rho -- 0.005 in the tested configuration --
+ * selects the fraction of tokens with the highest quantisation error for a
+ * residual correction).  The page names neither the error measure nor the
+ * correction; this library reads them as:
+ *   - per (batch, head), n = min(S, ceil(rho * S - 1e-3)) tokens (rho as
+ *     passed, a float; see jattn_repair_count) are repaired;
+ *   - a token's quantisation error is the e4m3 error bound of its key and
+ *     value rows, which grows with their magnitude: the n largest
+ *     |k_j|^2 + |v_j|^2 (fp32, rotated / normalised key before quantisation)
+ *     are taken, ties to the lower token index;
+ *   - a repaired token enters the attention with its exact key and value and
+ *     the logit of the 16-bit (fp16) query and key; every other token with
+ *     the e4m3 operands.  One softmax over all S keys.
+ * The whole path in one call, on `stream`:
+ *   prologue (as jattn_rope_qkv_norm / jattn_rope_qkv with JATTN_E4M3, plus
+ *   fp16 Q and the scores) -> selection -> exact fp16 keys / values of the
+ *   selected tokens -> FP8 attention over the other keys -> fp16 attention
+ *   over the selected keys, merged into o (and lse) through the two partial
+ *   log-sum-exps.
+ *   qkv_*, pos, theta, split : as jattn_rope_qkv.
+ *   norm_w, eps : query/key RMSNorm as jattn_rope_qkv_norm, or norm_w = NULL.
+ *   rho        : 0 <= rho <= 1 (0: plain FP8 path, nothing repaired).
+ *   workspace  : device scratch of at least
+ *                jattn_fwd_fp8_repair_workspace(shape, rho) bytes, 256-byte
+ *                aligned, owned by the caller; contents undefined afterwards.
+ *   o, lse, softmax_scale : as jattn_fwd_fp8.
+ *   repaired   : NULL, or int32 [B][H][n]: the repaired token indices (in
+ *                index order) are written there.
+ * Errors: as jattn_rope_qkv and jattn_fwd_fp8; JATTN_ERR_INVALID_ARG for rho
+ * outside [0, 1], a NULL or too small workspace; JATTN_ERR_ALIGNMENT for a
+ * workspace not 256-byte aligned.
+ */
+int32_t jattn_repair_count(const jattn_shape* shape, float rho);   /* n; -1 on invalid arguments */
+size_t jattn_fwd_fp8_repair_workspace(const jattn_shape* shape, float rho);   /* 0 on invalid arguments */
+jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                  const void* qkv_ref, const int32_t* pos, float theta,
+                                  const int32_t split[3], const float* norm_w, float eps, float rho,
+                                  void* workspace, size_t workspace_bytes, void* o, float* lse,
+                                  int32_t* repaired, float softmax_scale, void* stream);
+
+/*
  * Synchronise `stream`, read the current device's status word and return
  * JATTN_OK, JATTN_ERR_INTERNAL, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (in
  * that order of precedence).  The raw

@@ -105,6 +105,42 @@ def test_rope_norm_rejects_bad_arguments():
     assert f(*args(A, 1e-6, _split(16, 56, 58))) == jattn.ERR_INVALID_ARG
 
 
+def test_repair_count_and_workspace_on_the_host():
+    """Pure host arithmetic: n = ceil(rho * S - 1e-3) within [0, S]; the
+    workspace grows with S and n; invalid arguments give -1 / 0."""
+    lib = jattn.load()
+    assert lib.jattn_repair_count(shape(B=2, H=24, St=512, Si=16384), 0.005) == 85
+    assert lib.jattn_repair_count(shape(St=10), 0.3) == 3
+    assert lib.jattn_repair_count(shape(St=10), 0.0) == 0
+    assert lib.jattn_repair_count(shape(St=10), 1.0) == 10
+    assert lib.jattn_repair_count(shape(St=10), 1.5) == -1
+    assert lib.jattn_repair_count(shape(d=96), 0.1) == -1
+    w0 = lib.jattn_fwd_fp8_repair_workspace(shape(St=300), 0.0)
+    w1 = lib.jattn_fwd_fp8_repair_workspace(shape(St=300), 0.1)
+    assert 0 < w0 < w1 and w1 % 256 == 0
+    assert lib.jattn_fwd_fp8_repair_workspace(shape(St=300), -0.1) == 0
+
+
+def test_repair_rejects_bad_arguments():
+    lib = jattn.load()
+    f = lib.jattn_fwd_fp8_repair
+    sp = _split(16, 56, 56)
+    need = lib.jattn_fwd_fp8_repair_workspace(shape(), 0.1)
+
+    def call(rho=0.1, ws=A, nbytes=None, o=A, norm=None, eps=1e-6, rep=None, split=sp):
+        return f(shape(), A, None, None, A, 1e4, split, norm, eps, rho, ws, need if nbytes is None else nbytes,
+                 o, None, rep, 0.0, None)
+    assert call(rho=1.5) == jattn.ERR_INVALID_ARG
+    assert call(rho=float("nan")) == jattn.ERR_INVALID_ARG
+    assert call(ws=None) == jattn.ERR_INVALID_ARG
+    assert call(o=None) == jattn.ERR_INVALID_ARG
+    assert call(nbytes=need - 1) == jattn.ERR_INVALID_ARG
+    assert call(ws=A + 16) == jattn.ERR_ALIGNMENT
+    assert call(norm=A, eps=0.0) == jattn.ERR_INVALID_ARG
+    assert call(rep=A + 2) == jattn.ERR_ALIGNMENT
+    assert call(split=_split(16, 56, 58)) == jattn.ERR_INVALID_ARG
+
+
 def test_quant_rejects_bad_arguments():
     lib = jattn.load()
     f = lib.jattn_quant_fp8
