@@ -1,0 +1,53 @@
+// FP8 attention with token repair for callers that cannot allocate device
+// memory: the same path as jattn_fwd_fp8_repair, with its workspace in a
+// file-scope device array instead of a caller buffer.
+//
+// The array lives in this translation unit alone, so (with the CUDA
+// runtime's default lazy module loading) its memory is reserved only once a
+// process first calls this entry point on a device.  Its address is looked
+// up once per device and cached.  Calls on one device share the array: they
+// must not overlap in time (one stream, or serialised by the caller).
+#include <cstdint>
+#include <mutex>
+#include <cuda_runtime.h>
+
+#include "jattn.h"
+
+namespace {
+
+constexpr size_t kScratchBytes = JATTN_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) uint8_t g_repair_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_addr[kMaxDevices] = {};
+
+void* scratch_address() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_repair_scratch) != cudaSuccess) return nullptr;
+    g_addr[dev] = p;
+  }
+  return g_addr[dev];
+}
+
+}  // namespace
+
+extern "C" jattn_status jattn_fwd_fp8_repair_noalloc(const jattn_shape* shape, const void* qkv_txt,
+                                                     const void* qkv_img, const void* qkv_ref, const int32_t* pos,
+                                                     float theta, const int32_t split[3], const float* norm_w,
+                                                     float eps, float rho, void* o, float* lse, int32_t* repaired,
+                                                     float softmax_scale, void* stream) {
+  const size_t need = jattn_fwd_fp8_repair_workspace(shape, rho);
+  if (need == 0)   // invalid shape or rho: the full entry point reports which, before any launch
+    return jattn_fwd_fp8_repair(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, norm_w, eps, rho, nullptr, 0,
+                                o, lse, repaired, softmax_scale, stream);
+  if (need > kScratchBytes) return JATTN_ERR_UNSUPPORTED;
+  void* ws = scratch_address();
+  if (ws == nullptr) return JATTN_ERR_CUDA;
+  return jattn_fwd_fp8_repair(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, norm_w, eps, rho, ws,
+                              kScratchBytes, o, lse, repaired, softmax_scale, stream);
+}

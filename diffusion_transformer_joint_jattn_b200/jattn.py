@@ -34,7 +34,7 @@ _CODE_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, E4M3: torch.float8_e4m
 _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 
 SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_fp8_repair",
-           "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_bf16", "jattn_fwd_fp8",
+           "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc", "jattn_fwd_bf16", "jattn_fwd_fp8",
            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -71,6 +71,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                          ctypes.c_size_t, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8_repair_workspace.argtypes = [sp, f32]
     lib.jattn_repair_count.argtypes = [sp, f32]
+    lib.jattn_fwd_fp8_repair_noalloc.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, f32, vp, vp,
+                                                 vp, f32, vp]
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
@@ -297,6 +299,35 @@ def fwd_fp8_repair(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: 
     if want_repaired:
         out.append(rep)
     return out[0] if len(out) == 1 else tuple(out)
+
+
+NOALLOC_SCRATCH_BYTES = 640 << 20
+
+
+def fwd_fp8_repair_noalloc(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], o, theta: float = 10000.0,
+                           rho: float = 0.005, norm_w=None, eps: float = 1e-6, lse=None, repaired=None,
+                           softmax_scale: float = 0.0, stream=None):
+    """jattn_fwd_fp8_repair_noalloc: the FP8-with-repair path with the
+    library's own device scratch.  The caller passes every output buffer
+    (o bf16 [B, S, H, d]; optional lse fp32 [B, H, S] and repaired int32
+    [B, H, n]); nothing is allocated here or in the library."""
+    lib = load()
+    parts = [qkv_txt, qkv_img, qkv_ref]
+    ref = next(t for t in parts if t is not None)
+    B, _, _, H, d = ref.shape
+    lens = [0 if t is None else t.shape[1] for t in parts]
+    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
+        if t is not None:
+            _dev(t, name, torch.bfloat16)
+    _dev(pos, "pos", torch.int32)
+    _dev(o, "o", torch.bfloat16)
+    sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
+    shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
+    _check(lib.jattn_fwd_fp8_repair_noalloc(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref),
+                                            _ptr(pos), float(theta), sp, _ptr(norm_w), float(eps), float(rho), _ptr(o),
+                                            _ptr(lse), _ptr(repaired), float(softmax_scale), _stream(stream)),
+           "jattn_fwd_fp8_repair_noalloc")
+    return o
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",

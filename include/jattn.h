@@ -204,6 +204,27 @@ jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt,
                                   int32_t* repaired, float softmax_scale, void* stream);
 
 /*
+ * jattn_fwd_fp8_repair for callers that cannot allocate device memory: the
+ * workspace is a file-scope device array of JATTN_NOALLOC_SCRATCH_BYTES
+ * inside the library, reserved when a process first calls this function on a
+ * device (its address is looked up once per device).  The library makes no
+ * allocation on this path.
+ *   Arguments: as jattn_fwd_fp8_repair without workspace / workspace_bytes.
+ *   Errors: as jattn_fwd_fp8_repair; JATTN_ERR_UNSUPPORTED when
+ *   jattn_fwd_fp8_repair_workspace(shape, rho) exceeds the array (checked
+ *   before anything is launched), JATTN_ERR_CUDA if the array cannot be
+ *   mapped.
+ *   Calls on one device share the array: they must not overlap in time (use
+ *   one stream per device, or serialise).
+ */
+#define JATTN_NOALLOC_SCRATCH_BYTES ((size_t)640 << 20)
+jattn_status jattn_fwd_fp8_repair_noalloc(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                          const void* qkv_ref, const int32_t* pos, float theta,
+                                          const int32_t split[3], const float* norm_w, float eps, float rho,
+                                          void* o, float* lse, int32_t* repaired, float softmax_scale,
+                                          void* stream);
+
+/*
  * Synchronise `stream`, read the current device's status word and return
  * JATTN_OK, JATTN_ERR_INTERNAL, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (in
  * that order of precedence).  The raw

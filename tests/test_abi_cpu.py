@@ -141,6 +141,20 @@ def test_repair_rejects_bad_arguments():
     assert call(split=_split(16, 56, 58)) == jattn.ERR_INVALID_ARG
 
 
+def test_noalloc_refuses_before_launch():
+    """The allocation-free entry point: an input whose workspace exceeds the
+    library's scratch array is refused on the host, and invalid shapes or
+    budgets give the same codes as the workspace entry point."""
+    lib = jattn.load()
+    f = lib.jattn_fwd_fp8_repair_noalloc
+    sp = _split(16, 56, 56)
+    big = shape(B=2, H=24, St=512, Si=16384 * 2)            # ~1 GB of workspace
+    assert lib.jattn_fwd_fp8_repair_workspace(big, 0.005) > jattn.NOALLOC_SCRATCH_BYTES
+    assert f(big, A, A, None, A, 1e4, sp, None, 1e-6, 0.005, A, None, None, 0.0, None) == jattn.ERR_UNSUPPORTED
+    assert f(shape(), A, None, None, A, 1e4, sp, None, 1e-6, 1.5, A, None, None, 0.0, None) == jattn.ERR_INVALID_ARG
+    assert f(shape(d=96), A, None, None, A, 1e4, sp, None, 1e-6, 0.1, A, None, None, 0.0, None) == jattn.ERR_UNSUPPORTED
+
+
 def test_quant_rejects_bad_arguments():
     lib = jattn.load()
     f = lib.jattn_quant_fp8
