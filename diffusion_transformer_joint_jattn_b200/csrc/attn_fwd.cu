@@ -323,8 +323,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
     // exceeds the e4m3 range while p <= 2^8.
     const float p8_log2 = 8.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
+    // FP8: the K / V block scales of the next tile are fetched one tile ahead
+    // so that their load latency stays off the S -> P chain.
+    float sk_nxt = 0.f, sv_nxt = 0.f;
+    if constexpr (FP8) {
+      sk_nxt = sc_k[0];
+      sv_nxt = sc_v[0];
+    }
 
     for (int j = 0; j < n_kv; ++j) {
+      float c_j = sl2, bias = 0.f;
+      if constexpr (FP8) {
+        c_j = sl2 * sq * sk_nxt;
+        bias = __log2f(sv_nxt / max_sv) + p8_log2;
+        if (j + 1 < n_kv) {
+          sk_nxt = sc_k[j + 1];
+          sv_nxt = sc_v[j + 1];
+        }
+      }
       // Keys left out of this pass (same for every row of the tile).
       uint4 km = make_uint4(0u, 0u, 0u, 0u);
       if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * n_kv + j);
@@ -340,11 +356,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(r[e]);
       }
 
-      float c_j = sl2, bias = 0.f;
-      if constexpr (FP8) {
-        c_j = sl2 * sq * sc_k[j];
-        bias = __log2f(sc_v[j] / max_sv) + p8_log2;
-      }
       const int valid = p.S_kv - j * BN;
       if (valid < BN) {
 #pragma unroll

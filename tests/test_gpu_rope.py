@@ -220,3 +220,28 @@ def test_rope_full_size_2048(cuda_device):
     vr = qkv[..., 2, :, :].permute(0, 2, 1, 3).to(torch.float32).numpy()
     _, sv = oracle.quantize_blocks(vr)
     np.testing.assert_array_equal(sc[2].cpu().numpy(), sv)
+
+
+@pytest.mark.slow
+def test_rope_norm_full_size_2048(cuda_device):
+    """The fused query/key RMSNorm at the full 2048x2048 size (S = 16896),
+    sampled tokens: 16-bit within the norm's bound."""
+    w = W.BY_NAME["t2i_2048_base"]
+    inp = W.make_inputs(w, 0)
+    nw = W.norm_weights(w.d, 0)
+    dinp = to_device(inp, cuda_device)
+    q, k, v, _ = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                                "fp16", norm_w=nw.to(cuda_device), eps=1e-6)
+    torch.cuda.synchronize()
+    toks = W.sample_rows(w.with_batch_heads(B=1, H=1), 512, seed=9)[0, 0]
+    qkv = torch.cat([inp["qkv_txt"], inp["qkv_img"]], dim=1)
+    stream = (toks >= w.S_txt).long().numpy()                           # 0 = txt, 1 = img
+    for b in range(w.B):
+        x = qkv[b, toks].to(torch.float64).numpy()                      # [m, 3, H, d]
+        pos = inp["pos"][toks].numpy()
+        for which, got in ((0, q), (1, k)):
+            wv = nw.to(torch.float64).numpy()[stream, which]            # [m, d]
+            xn = oracle.rms_norm(np.transpose(x[:, which], (1, 0, 2)), wv[None], 1e-6)
+            xr = oracle.rope_rotate(xn, pos, w.split, w.theta)
+            _check_rotated(got[b][:, toks], xr, torch.float16, "qk"[which], rel=2.0 ** -18)
+    assert jattn.device_status()[0] == jattn.OK
