@@ -34,7 +34,8 @@ _CODE_DTYPE = {BF16: torch.bfloat16, FP16: torch.float16, E4M3: torch.float8_e4m
 _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 
 SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_fp8_repair",
-           "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc", "jattn_fwd_bf16", "jattn_fwd_fp8",
+           "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc",
+           "jattn_joint_attention_host", "jattn_joint_attention_host_workspace", "jattn_fwd_bf16", "jattn_fwd_fp8",
            "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -71,6 +72,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                          ctypes.c_size_t, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8_repair_workspace.argtypes = [sp, f32]
     lib.jattn_repair_count.argtypes = [sp, f32]
+    lib.jattn_joint_attention_host.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), i32, vp, f32, vp,
+                                               ctypes.c_size_t, vp]
+    lib.jattn_joint_attention_host_workspace.argtypes = [sp, i32]
     lib.jattn_fwd_fp8_repair_noalloc.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, f32, vp, vp,
                                                  vp, f32, vp]
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
@@ -84,6 +88,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         if name not in ("jattn_status_string", "jattn_version"):
             getattr(lib, name).restype = i32
     lib.jattn_fwd_fp8_repair_workspace.restype = ctypes.c_size_t
+    lib.jattn_joint_attention_host_workspace.restype = ctypes.c_size_t
     _lib = lib
     return lib
 
@@ -332,22 +337,49 @@ def fwd_fp8_repair_noalloc(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int],
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
                     operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None,
-                    norm_w=None, eps: float = 1e-6):
+                    norm_w=None, eps: float = 1e-6, workspace=None):
     """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8),
     with the query/key RMSNorm fused into rope_qkv when ``norm_w`` is given.
 
-    Accepts CUDA tensors, or CPU tensors (then copied to the current device
-    -- asynchronously when they are pinned -- and the output copied back,
-    into ``out`` if given, e.g. a pinned bf16 [B, S, H, d] buffer).
-    Returns O bf16 [B, S, H, d] (and LSE)."""
+    CUDA tensors: the device entry points, asynchronous on ``stream``.
+    CPU tensors (pinned for overlap): jattn_joint_attention_host, which
+    copies in, runs the path and copies O out pipelined over the batch; the
+    result lands in ``out`` (a bf16 [B, S, H, d] host tensor, allocated here
+    if None) and the call returns once it is there.  The host entry has no
+    LSE output and no norm; those need device tensors.
+    Returns O bf16 [B, S, H, d] (and LSE for device tensors)."""
     parts = [qkv_txt, qkv_img, qkv_ref]
-    on_host = not next(t for t in parts if t is not None).is_cuda
-    if on_host:
+    ref = next(t for t in parts if t is not None)
+    if not ref.is_cuda:
+        if want_lse or norm_w is not None:
+            raise ValueError("LSE output and the query/key norm need device tensors")
+        lib = load()
+        B, _, _, H, d = ref.shape
+        lens = [0 if t is None else t.shape[1] for t in parts]
+        for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
+            if t is not None and (t.dtype != torch.bfloat16 or not t.is_contiguous()):
+                raise ValueError(f"{name} must be a contiguous bf16 tensor")
+        if pos.dtype != torch.int32 or not pos.is_contiguous():
+            raise ValueError("pos must be a contiguous int32 tensor")
+        S = sum(lens)
+        code = E4M3 if path == "fp8" else _NAME_CODE[operand_dtype]
+        if path not in ("bf16", "fp8"):
+            raise ValueError(f"unknown path {path!r}")
+        shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
+        need = lib.jattn_joint_attention_host_workspace(ctypes.byref(shape), code)
         dev = torch.device("cuda", torch.cuda.current_device())
-        parts = [None if t is None else t.to(dev, non_blocking=True) for t in parts]
-        pos = pos.to(dev, non_blocking=True)
-        if norm_w is not None:
-            norm_w = norm_w.to(dev, non_blocking=True)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        if out is None:
+            out = torch.empty(B, S, H, d, dtype=torch.bfloat16).pin_memory()
+        sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
+        st = torch.cuda.current_stream() if stream is None else stream
+        _check(lib.jattn_joint_attention_host(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref),
+                                              _ptr(pos), float(theta), sp, code, _ptr(out), 0.0, _ptr(workspace),
+                                              workspace.numel() * workspace.element_size(),
+                                              ctypes.c_void_p(st.cuda_stream)), "jattn_joint_attention_host")
+        st.synchronize()
+        return out
     if path == "bf16":
         q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream, norm_w=norm_w, eps=eps)
         o, lse = fwd_bf16(q, k, v, want_lse=want_lse, stream=stream)
@@ -356,15 +388,6 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
         o, lse = fwd_fp8(q, k, v, sc, want_lse=want_lse, stream=stream)
     else:
         raise ValueError(f"unknown path {path!r}")
-    if on_host:
-        if out is not None:
-            out.copy_(o, non_blocking=out.is_pinned())
-            if out.is_pinned():
-                torch.cuda.current_stream().synchronize()
-            o = out
-        else:
-            o = o.to("cpu")
-        lse = None if lse is None else lse.to("cpu")
     return (o, lse) if want_lse else o
 
 

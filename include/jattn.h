@@ -225,6 +225,30 @@ jattn_status jattn_fwd_fp8_repair_noalloc(const jattn_shape* shape, const void* 
                                           void* stream);
 
 /*
+ * The whole path on HOST buffers, for callers whose inputs and outputs live
+ * in host memory: copies in, jattn_rope_qkv + jattn_fwd_bf16 (path JATTN_FP16
+ * or JATTN_BF16: the 16-bit operand type) or + jattn_fwd_fp8 (path
+ * JATTN_E4M3), copy of O out.  The work is pipelined over the batch: the
+ * copies of one batch entry overlap the kernels of another, on two copy
+ * streams the library creates once per host thread and device.  The call is
+ * ordered like one operation on `stream`: it starts after the work already
+ * enqueued there, and `stream` completes only after O is in host memory.
+ *   qkv_*, pos : HOST pointers, layouts as jattn_rope_qkv.  Page-locked
+ *                (pinned) memory lets the copies overlap the kernels;
+ *                pageable memory works but serialises them.
+ *   o          : HOST pointer, bf16 [B, S, H, d].
+ *   workspace  : DEVICE scratch of jattn_joint_attention_host_workspace()
+ *                bytes, 256-byte aligned, owned by the caller.
+ * Errors: as the device entry points, checked before anything is enqueued;
+ * JATTN_ERR_INVALID_ARG for a NULL or too small workspace.
+ */
+size_t jattn_joint_attention_host_workspace(const jattn_shape* shape, jattn_dtype path);   /* 0 if invalid */
+jattn_status jattn_joint_attention_host(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                                        const void* qkv_ref, const int32_t* pos, float theta,
+                                        const int32_t split[3], jattn_dtype path, void* o, float softmax_scale,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronise `stream`, read the current device's status word and return
  * JATTN_OK, JATTN_ERR_INTERNAL, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE (in
  * that order of precedence).  The raw

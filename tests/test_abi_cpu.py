@@ -155,6 +155,37 @@ def test_noalloc_refuses_before_launch():
     assert f(shape(d=96), A, None, None, A, 1e4, sp, None, 1e-6, 0.1, A, None, None, 0.0, None) == jattn.ERR_UNSUPPORTED
 
 
+def test_host_entry_workspace_and_argument_checks():
+    """jattn_joint_attention_host: the workspace size is host arithmetic
+    (inputs + laid-out operands + output, 256-byte segments); argument errors
+    come back before anything is enqueued."""
+    lib = jattn.load()
+    ws16 = lib.jattn_joint_attention_host_workspace(shape(B=2, St=100, Si=64), jattn.FP16)
+    ws8 = lib.jattn_joint_attention_host_workspace(shape(B=2, St=100, Si=64), jattn.E4M3)
+    S, H, d = 164, 1, 128
+    assert ws16 >= 2 * S * 3 * H * d * 2 + 3 * 2 * H * S * d * 2 + 2 * S * H * d * 2
+    assert 0 < ws8 < ws16 and ws16 % 256 == 0
+    assert lib.jattn_joint_attention_host_workspace(shape(d=96), jattn.FP16) == 0
+    f = lib.jattn_joint_attention_host
+    sp = _split(16, 56, 56)
+    need = lib.jattn_joint_attention_host_workspace(shape(), jattn.FP16)
+    ok = dict(sh=shape(), t=A, pos=A, split=sp, path=jattn.FP16, o=A, ws=A, n=need, theta=1e4)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["sh"], a["t"], None, None, a["pos"], a["theta"], a["split"], a["path"], a["o"], 0.0, a["ws"],
+                 a["n"], None)
+    assert call(path=9) == jattn.ERR_UNSUPPORTED
+    assert call(sh=shape(d=96)) == jattn.ERR_UNSUPPORTED
+    assert call(t=None) == jattn.ERR_INVALID_ARG
+    assert call(o=None) == jattn.ERR_INVALID_ARG
+    assert call(ws=None) == jattn.ERR_INVALID_ARG
+    assert call(n=need - 1) == jattn.ERR_INVALID_ARG
+    assert call(ws=A + 16) == jattn.ERR_ALIGNMENT
+    assert call(theta=0.0) == jattn.ERR_INVALID_ARG
+    assert call(split=_split(16, 56, 58)) == jattn.ERR_INVALID_ARG
+
+
 def test_quant_rejects_bad_arguments():
     lib = jattn.load()
     f = lib.jattn_quant_fp8

@@ -123,12 +123,40 @@ def test_joint_attention_with_qk_norm(cuda_device, case):
     assert jattn.device_status()[0] == jattn.OK
 
 
-def test_host_buffers_end_to_end(cuda_device):
-    """The public one-call API with host tensors: copies in, runs the path,
-    copies out; same result as the device-tensor call."""
+@pytest.mark.parametrize("pinned", [False, True])
+def test_host_buffers_end_to_end(cuda_device, pinned):
+    """The public one-call API with host tensors (jattn_joint_attention_host:
+    copies in, the path pipelined over the batch, copy out): the same bytes
+    as the device-tensor call, from pageable or pinned host memory."""
     w = W.BY_NAME["tiny"]
     inp = W.make_inputs(w, 0)
+    if pinned:
+        inp = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
     o_host = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
     assert o_host.device.type == "cpu"
     o_dev, _ = _run_bf16(w, inp, cuda_device, want_lse=False)
     assert torch.equal(o_host, o_dev.cpu())
+
+
+@pytest.mark.parametrize("path", ["bf16", "fp8"])
+def test_host_entry_pipelined_batch(cuda_device, path):
+    """B = 3 with a reference image: every batch entry runs as its own
+    (copy-in, kernels, copy-out) stage on the three streams; the result equals
+    the device entry points' on the whole batch, also when the caller's
+    stream already has work queued and the output buffer is reused."""
+    w = W.custom(B=3, H=2, d=128, S_txt=77, grid=9, n_ref=1)
+    inp = {k: (None if v is None else v.pin_memory()) for k, v in W.make_inputs(w, 5).items()}
+    d = to_device(inp, cuda_device)
+    if path == "bf16":
+        q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "fp16")
+        o_dev, _ = jattn.fwd_bf16(q, k, v)
+    else:
+        q, k, v, sc = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "e4m3")
+        o_dev, _ = jattn.fwd_fp8(q, k, v, sc)
+    out = torch.empty(w.B, w.S, w.H, w.d, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        torch.cuda._sleep(1000000)                 # work already queued on the caller's stream
+        o_host = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split,
+                                       w.theta, path=path, out=out)
+        assert torch.equal(o_host, o_dev.cpu())
+    assert jattn.device_status()[0] == jattn.OK
