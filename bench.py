@@ -34,7 +34,7 @@ WORKLOAD = "t2i_2048_base"
 # capture of the same kernel on t2i_1024_base (profiles/attn_fwd_t2i_1024_base.md,
 # dram__bytes_read.sum + dram__bytes_write.sum = 207.44 MB) scaled by the token
 # count 16896 / 4608 (the traffic is Q, K, V and O once each, linear in tokens).
-FWD_TRAFFIC_BYTES = 207.44e6 * 16896 / 4608
+FWD_TRAFFIC_BYTES = 206.96e6 * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 

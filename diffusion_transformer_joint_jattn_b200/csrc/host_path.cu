@@ -1,6 +1,9 @@
 // The whole path on host buffers: copies in, prologue + attention, copy out,
-// pipelined over the batch so that the host<->device copies of one batch
-// entry overlap the kernels of another.
+// pipelined over (batch entry, head group) chunks so that the host<->device
+// copies of one chunk overlap the kernels of another.  A head group is a
+// strided slice of the [B, S, 3, H, d] inputs and of the [B, S, H, d]
+// output, moved with 2-D copies into compact per-chunk device buffers, on
+// which the device entry points run with H = heads per group.
 //
 // Three streams: the caller's stream runs the kernels; a copy-in and a
 // copy-out stream (created once per thread and device, non-blocking) carry
@@ -45,12 +48,24 @@ Pipe* pipe_for_device() {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Heads per chunk: 2 (or 3) when that divides H, else all H.  Small chunks
+// keep the pipeline's fill and drain short (the first chunk's copy-in and the
+// last chunk's kernels and copy-out are not overlapped); at t2i_2048_base
+// (H = 24) 12 groups per batch entry run within 1 ms of the copy-in alone.
+int head_groups(int H) {
+  for (int hg : {2, 3})
+    if (H % hg == 0) return H / hg;
+  return 1;
+}
+
 struct HostLayout {
   size_t part[3], pos, q, k, v, scales, o, total;
 };
 
 bool valid_path(jattn_dtype path) { return path == JATTN_FP16 || path == JATTN_BF16 || path == JATTN_E4M3; }
 
+// Every chunk (b, g) owns a compact slice of each buffer; the slices tile
+// the buffers, so the sizes are those of the whole batch.
 HostLayout host_layout(const jattn_shape* s, jattn_dtype path) {
   const size_t B = s->B, H = s->H, d = s->d, S = static_cast<size_t>(s->S_txt) + s->S_img + s->S_ref;
   const size_t lens[3] = {static_cast<size_t>(s->S_txt), static_cast<size_t>(s->S_img),
@@ -117,14 +132,15 @@ extern "C" jattn_status jattn_joint_attention_host(const jattn_shape* shape, con
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const int B = shape->B, H = shape->H, d = shape->d;
+  const int G = head_groups(H), Hg = H / G;
   const int S = shape->S_txt + shape->S_img + shape->S_ref;
   const size_t eb = path == JATTN_E4M3 ? 1 : 2;
   const size_t nb = (static_cast<size_t>(S) + JATTN_BLOCK - 1) / JATTN_BLOCK;
-  const size_t qkv_b[3] = {static_cast<size_t>(lens[0]) * 3 * H * d * 2, static_cast<size_t>(lens[1]) * 3 * H * d * 2,
-                           static_cast<size_t>(lens[2]) * 3 * H * d * 2};
-  const size_t lay_b = static_cast<size_t>(H) * S * d * eb;       // one batch entry of q / k / v
-  const size_t out_b = static_cast<size_t>(S) * H * d * 2;
-  const jattn_shape one{1, H, shape->S_txt, shape->S_img, shape->S_ref, d};
+  const size_t row_in = static_cast<size_t>(H) * d * 2;          // host input: one (token, Q|K|V) row
+  const size_t row_grp = static_cast<size_t>(Hg) * d * 2;        // the group's part of it
+  const size_t lay_c = static_cast<size_t>(Hg) * S * d * eb;     // one chunk of laid-out q / k / v
+  const size_t out_c = static_cast<size_t>(S) * Hg * d * 2;      // one chunk of o
+  const jattn_shape one{1, Hg, shape->S_txt, shape->S_img, shape->S_ref, d};
 
 #define JATTN_CU(x) do { if ((x) != cudaSuccess) return JATTN_ERR_CUDA; } while (0)
   JATTN_CU(cudaEventRecord(P->start, cs));
@@ -132,41 +148,46 @@ extern "C" jattn_status jattn_joint_attention_host(const jattn_shape* shape, con
   JATTN_CU(cudaStreamWaitEvent(P->out, P->start, 0));
   JATTN_CU(cudaMemcpyAsync(ws + L.pos, pos, static_cast<size_t>(S) * 3 * 4, cudaMemcpyHostToDevice, P->in));
   for (int b = 0; b < B; ++b) {
-    const void* dparts[3] = {nullptr, nullptr, nullptr};
-    for (int i = 0; i < 3; ++i) {
-      if (lens[i] == 0) continue;
-      uint8_t* dst = ws + L.part[i] + b * qkv_b[i];
-      JATTN_CU(cudaMemcpyAsync(dst, static_cast<const uint8_t*>(parts[i]) + b * qkv_b[i], qkv_b[i],
-                               cudaMemcpyHostToDevice, P->in));
-      dparts[i] = dst;
+    for (int g = 0; g < G; ++g) {
+      const size_t c = static_cast<size_t>(b) * G + g;           // chunk index
+      const void* dparts[3] = {nullptr, nullptr, nullptr};
+      for (int i = 0; i < 3; ++i) {
+        if (lens[i] == 0) continue;
+        const size_t rows = static_cast<size_t>(lens[i]) * 3;     // (token, Q|K|V) rows of this stream
+        uint8_t* dst = ws + L.part[i] + c * rows * row_grp;
+        const uint8_t* src = static_cast<const uint8_t*>(parts[i]) + b * rows * row_in + g * row_grp;
+        JATTN_CU(cudaMemcpy2DAsync(dst, row_grp, src, row_in, row_grp, rows, cudaMemcpyHostToDevice, P->in));
+        dparts[i] = dst;
+      }
+      JATTN_CU(cudaEventRecord(P->ready, P->in));
+      JATTN_CU(cudaStreamWaitEvent(cs, P->ready, 0));
+      void* q = ws + L.q + c * lay_c;
+      void* k = ws + L.k + c * lay_c;
+      void* v = ws + L.v + c * lay_c;
+      void* oc = ws + L.o + c * out_c;
+      const int32_t* dpos = reinterpret_cast<const int32_t*>(ws + L.pos);
+      jattn_status st;
+      if (path == JATTN_E4M3) {
+        float* sc = reinterpret_cast<float*>(ws + L.scales) + c * 3 * Hg * nb;
+        st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], dpos, theta, split, JATTN_E4M3, q, k, v, sc, cs);
+        if (st == JATTN_OK) st = jattn_fwd_fp8(&one, q, k, v, sc, oc, nullptr, softmax_scale, cs);
+      } else {
+        st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], dpos, theta, split, path, q, k, v, nullptr, cs);
+        if (st == JATTN_OK) st = jattn_fwd_bf16(&one, path, q, k, v, oc, nullptr, softmax_scale, cs);
+      }
+      if (st != JATTN_OK) return st;
+      JATTN_CU(cudaEventRecord(P->done, cs));
+      JATTN_CU(cudaStreamWaitEvent(P->out, P->done, 0));
+      // o chunk [S][Hg][d] -> host o[b][s][g*Hg .. g*Hg+Hg)[d]
+      uint8_t* dst = static_cast<uint8_t*>(o) + static_cast<size_t>(b) * S * row_in + g * row_grp;
+      JATTN_CU(cudaMemcpy2DAsync(dst, row_in, oc, row_grp, row_grp, S, cudaMemcpyDeviceToHost, P->out));
     }
-    JATTN_CU(cudaEventRecord(P->ready, P->in));
-    JATTN_CU(cudaStreamWaitEvent(cs, P->ready, 0));
-    void* q = ws + L.q + b * lay_b;
-    void* k = ws + L.k + b * lay_b;
-    void* v = ws + L.v + b * lay_b;
-    void* ob = ws + L.o + b * out_b;
-    jattn_status st;
-    if (path == JATTN_E4M3) {
-      float* sc = reinterpret_cast<float*>(ws + L.scales) + static_cast<size_t>(b) * 3 * H * nb;
-      st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], reinterpret_cast<const int32_t*>(ws + L.pos), theta,
-                          split, JATTN_E4M3, q, k, v, sc, cs);
-      if (st == JATTN_OK) st = jattn_fwd_fp8(&one, q, k, v, sc, ob, nullptr, softmax_scale, cs);
-    } else {
-      st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], reinterpret_cast<const int32_t*>(ws + L.pos), theta,
-                          split, path, q, k, v, nullptr, cs);
-      if (st == JATTN_OK) st = jattn_fwd_bf16(&one, path, q, k, v, ob, nullptr, softmax_scale, cs);
-    }
-    if (st != JATTN_OK) return st;
-    JATTN_CU(cudaEventRecord(P->done, cs));
-    JATTN_CU(cudaStreamWaitEvent(P->out, P->done, 0));
-    JATTN_CU(cudaMemcpyAsync(static_cast<uint8_t*>(o) + b * out_b, ob, out_b, cudaMemcpyDeviceToHost, P->out));
   }
   JATTN_CU(cudaEventRecord(P->copied, P->out));
   JATTN_CU(cudaStreamWaitEvent(cs, P->copied, 0));
-  // The copy-in stream must not run ahead into a later call's copies while
-  // this call's kernels still read the inputs: later calls start by waiting
-  // on the caller's stream, which now includes everything above.
+  // A later call starts by waiting on the caller's stream, which now
+  // includes everything above, so its copies cannot overrun this call's
+  // kernels.
 #undef JATTN_CU
   return JATTN_OK;
 }

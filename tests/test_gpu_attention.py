@@ -138,13 +138,15 @@ def test_host_buffers_end_to_end(cuda_device, pinned):
     assert torch.equal(o_host, o_dev.cpu())
 
 
-@pytest.mark.parametrize("path", ["bf16", "fp8"])
-def test_host_entry_pipelined_batch(cuda_device, path):
-    """B = 3 with a reference image: every batch entry runs as its own
-    (copy-in, kernels, copy-out) stage on the three streams; the result equals
+@pytest.mark.parametrize("path,B,H", [("bf16", 3, 2), ("fp8", 3, 2), ("bf16", 2, 12), ("fp8", 1, 9),
+                                      ("bf16", 2, 5)])
+def test_host_entry_pipelined_batch(cuda_device, path, B, H):
+    """Every (batch entry, head group) chunk runs as its own (2-D copy in,
+    kernels, 2-D copy out) stage on the three streams -- H = 12 splits into
+    6 groups of 2 heads, 9 into 3 groups of 3, 2 and 5 stay whole; the result equals
     the device entry points' on the whole batch, also when the caller's
     stream already has work queued and the output buffer is reused."""
-    w = W.custom(B=3, H=2, d=128, S_txt=77, grid=9, n_ref=1)
+    w = W.custom(B=B, H=H, d=128, S_txt=77, grid=9, n_ref=1)
     inp = {k: (None if v is None else v.pin_memory()) for k, v in W.make_inputs(w, 5).items()}
     d = to_device(inp, cuda_device)
     if path == "bf16":
