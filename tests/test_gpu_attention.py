@@ -162,3 +162,44 @@ def test_host_entry_pipelined_batch(cuda_device, path, B, H):
                                        w.theta, path=path, out=out)
         assert torch.equal(o_host, o_dev.cpu())
     assert jattn.device_status()[0] == jattn.OK
+
+
+def test_cuda_graph_capture_and_replay(cuda_device):
+    """The device entry points enqueue work only (no allocation, no host
+    synchronisation), so the prologue + forward pair can be captured into a
+    CUDA graph and replayed: the replay gives the eager result, also after
+    the inputs change in place."""
+    w = W.custom(B=1, H=2, d=128, S_txt=40, grid=12, n_ref=0)
+    inp = W.make_inputs(w, 3)
+    d = to_device(inp, cuda_device)
+    q = torch.empty(w.B, w.H, w.S, w.d, dtype=torch.float16, device=cuda_device)
+    bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
+    o = torch.empty(w.B, w.S, w.H, w.d, dtype=torch.bfloat16, device=cuda_device)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+
+    def step():
+        jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], None, d["pos"], w.split, w.theta, "fp16", out=bufs, stream=s)
+        jattn.fwd_bf16(bufs[0], bufs[1], bufs[2], o=o, stream=s)
+
+    with torch.cuda.stream(s):
+        step()                                            # warm-up: module loading, tensor maps
+    torch.cuda.synchronize()
+    eager = o.clone()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step()
+    o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, eager)
+    d["qkv_img"].mul_(0.5)                                # new inputs, same buffers
+    g.replay()
+    torch.cuda.synchronize()
+    replayed = o.clone()
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.synchronize()
+    assert torch.equal(replayed, o)
+    assert not torch.equal(replayed, eager)
+    assert jattn.device_status()[0] == jattn.OK
