@@ -367,7 +367,7 @@ def measure_e2e(jattn, w, inp, dev, stream, steps, warmup, flops, world, max_ove
     return {"value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "api": "jattn.joint_attention -> jattn_joint_attention_host (C ABI, pinned host in/out, "
-                   "copies pipelined over the batch on copy streams)"}
+                   "copies pipelined with the kernels in (batch entry, 2-head) chunks on copy streams)"}
 
 
 def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
