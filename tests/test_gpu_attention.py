@@ -203,3 +203,29 @@ def test_cuda_graph_capture_and_replay(cuda_device):
     assert torch.equal(replayed, o)
     assert not torch.equal(replayed, eager)
     assert jattn.device_status()[0] == jattn.OK
+
+
+@pytest.mark.slow
+def test_long_sequence_and_wide_grid(cuda_device):
+    """Sizes far from the workloads: S = 65613 (513 key tiles, ragged tail;
+    256 sampled rows per head against the oracle) and B*H = 1600 small heads
+    (grid.y = 1600, every row checked)."""
+    w = W.custom(B=1, H=2, d=128, S_txt=77, grid=256, n_ref=0)            # S = 77 + 65536
+    inp = W.make_inputs(w, 2)
+    o, lse = _run_bf16(w, inp, cuda_device)
+    rows = W.sample_rows(w, 256, 2)
+    O, L = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], None, inp["pos"], w.split, w.theta, rows=rows,
+                                  workers=4)
+    got = gather_rows(o, rows)
+    assert rel_l2(got, O) <= BF16_REL_L2
+    assert max_abs(got, O) <= BF16_MAX_ABS
+    np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=2e-3, atol=5e-3)
+    w2 = W.custom(B=40, H=40, d=64, S_txt=5, grid=11, n_ref=0)           # S = 126 < one tile
+    inp2 = W.make_inputs(w2, 3)
+    o2, _ = _run_bf16(w2, inp2, cuda_device, want_lse=False)
+    O2, _ = oracle.joint_attention(inp2["qkv_txt"], inp2["qkv_img"], None, inp2["pos"], w2.split, w2.theta,
+                                   workers=4)
+    got2 = gather_rows(o2, torch.arange(w2.S).expand(w2.B, w2.H, w2.S))
+    assert rel_l2(got2, O2) <= BF16_REL_L2
+    assert max_abs(got2, O2) <= BF16_MAX_ABS
+    assert jattn.device_status()[0] == jattn.OK
