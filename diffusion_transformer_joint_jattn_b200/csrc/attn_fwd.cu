@@ -15,7 +15,9 @@
 //               epilogue O / l -> bf16 [B, S, H, d].
 //   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j.
 //               Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): each
-//               tile's softmax overlaps the other tile's tensor work.
+//               tile's softmax overlaps the other tile's tensor work.  With
+//               e4m3 operands P is handed over in two halves of 64 keys, so
+//               the first half's P.V overlaps the second half's softmax.
 //   warp 9      TMA producer: Q tiles once, K_j / V_j into smem rings.
 //   (warps 10, 11 idle: they complete the third warpgroup.)
 // The block starts at 168 registers per thread (384 x 168 = 64512); the
@@ -75,6 +77,7 @@ struct __align__(8) Bars {
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full[NQ], p_full[NQ], o_final[NQ];
+  uint64_t p_half[NQ];            // FP8: P of the tile's first 64 keys is in TMEM
   uint64_t mma_final;
   uint32_t tmem_base;
   uint32_t abort;
@@ -173,6 +176,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     for (int t = 0; t < NQ; ++t) {
       mbar_init(&bar->s_full[t], 1);
       mbar_init(&bar->p_full[t], BM);
+      mbar_init(&bar->p_half[t], BM);
       mbar_init(&bar->o_final[t], 1);
     }
     mbar_init(&bar->mma_final, 1);
@@ -242,10 +246,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
         any_mma = true;
       };
-      auto issue_pv = [&](int t, int vs, bool acc) {
+      auto issue_pv = [&](int t, int vs, bool acc, int kk0, int kk1) {
         const uint32_t vbase = sVa + vs * C::TB;
 #pragma unroll
-        for (int kk = 0; kk < C::PV_STEPS; ++kk) {
+        for (int kk = kk0; kk < kk1; ++kk) {
           const uint64_t bdesc = smem_desc(vbase + kk * C::MK * C::SWB, C::BOXB, 8 * C::SWB, C::SWMODE);
           if constexpr (FP8) mma_f8_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, acc || kk > 0);
           else mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, acc || kk > 0);
@@ -265,10 +269,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const bool more = j + 1 < n_kv;
           ok = mbar_wait(&bar->v_full[vs], (j / C::VS) & 1, ctl);
           for (int t = 0; t < NQ && ok; ++t) {
-            ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, vs, j > 0);
+            if constexpr (FP8) {
+              // P arrives in two halves: the first half's P.V steps overlap
+              // the softmax of the second half.
+              ok = mbar_wait(&bar->p_half[t], j & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, vs, j > 0, 0, C::PV_STEPS / 2);
+              ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, vs, true, C::PV_STEPS / 2, C::PV_STEPS);
+            } else {
+              ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
+              if (!ok) break;
+              tc_fence_after();
+              issue_pv(t, vs, j > 0, 0, C::PV_STEPS);
+            }
             if (t == NQ - 1) mma_commit(&bar->v_empty[vs]);
             if (more) {
               if (t == 0) {
@@ -407,18 +424,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
       if constexpr (FP8) {
-        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float2 x0 = __ffma2_rn(make_float2(v[4 * c + 0], v[4 * c + 1]), c2, nm2);
-          const float2 x1 = __ffma2_rn(make_float2(v[4 * c + 2], v[4 * c + 3]), c2, nm2);
-          const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
-          const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
-          acc0 = __fadd2_rn(acc0, e0);
-          acc1 = __fadd2_rn(acc1, e1);
-          pk[c] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int e = half * 64 + 4 * c;
+            const float2 x0 = __ffma2_rn(make_float2(v[e + 0], v[e + 1]), c2, nm2);
+            const float2 x1 = __ffma2_rn(make_float2(v[e + 2], v[e + 3]), c2, nm2);
+            const float2 e0 = make_float2(ex2_approx(x0.x), ex2_approx(x0.y));
+            const float2 e1 = make_float2(ex2_approx(x1.x), ex2_approx(x1.y));
+            acc0 = __fadd2_rn(acc0, e0);
+            acc1 = __fadd2_rn(acc1, e1);
+            pk[c] = pack_e4m3x4(e0.x, e0.y, e1.x, e1.y);
+          }
+          tmem_st16(ts + half * 16, pk);
+          if (half == 0) {
+            tc_fence_before();
+            mbar_arrive(&bar->p_half[t]);
+          }
         }
-        tmem_st32(ts, pk);
       } else {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
