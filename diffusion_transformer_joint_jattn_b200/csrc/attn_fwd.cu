@@ -379,23 +379,38 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < BN; ++e)
           if (e >= valid) v[e] = -INFINITY;
       }
+      auto row_max = [&]() {
+        float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
+#pragma unroll
+        for (int e = 4; e < BN - 4; e += 8) {
+          mx0 = max3(mx0, v[e + 0], v[e + 1]);
+          mx1 = max3(mx1, v[e + 2], v[e + 3]);
+          mx2 = max3(mx2, v[e + 4], v[e + 5]);
+          mx3 = max3(mx3, v[e + 6], v[e + 7]);
+        }
+        mx0 = max3(mx0, v[BN - 4], v[BN - 3]);
+        mx1 = max3(mx1, v[BN - 2], v[BN - 1]);
+        return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      };
+      float mx_raw = row_max();
+      // Keys left out of this pass hold zero codes (their logits are exactly
+      // 0, their values 0).  Where the row max is positive they cannot be the
+      // max, and their probabilities -- exp2(neg_m) each -- are taken off the
+      // row sum below.  Only a warp with a row whose max may be such a zero
+      // sets them to -inf one by one.
+      float n_left_out = 0.f;
       if ((km.x | km.y | km.z | km.w) != 0u) {
-        const uint32_t kw[4] = {km.x, km.y, km.z, km.w};
+        if (__any_sync(0xffffffffu, !(mx_raw > 0.f))) {
+          const uint32_t kw[4] = {km.x, km.y, km.z, km.w};
 #pragma unroll
-        for (int e = 0; e < BN; ++e)
-          if ((kw[e >> 5] >> (e & 31)) & 1u) v[e] = -INFINITY;
+          for (int e = 0; e < BN; ++e)
+            if ((kw[e >> 5] >> (e & 31)) & 1u) v[e] = -INFINITY;
+          mx_raw = row_max();
+        } else {
+          n_left_out = static_cast<float>(__popc(km.x) + __popc(km.y) + __popc(km.z) + __popc(km.w));
+        }
       }
-      float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
-#pragma unroll
-      for (int e = 4; e < BN - 4; e += 8) {
-        mx0 = max3(mx0, v[e + 0], v[e + 1]);
-        mx1 = max3(mx1, v[e + 2], v[e + 3]);
-        mx2 = max3(mx2, v[e + 4], v[e + 5]);
-        mx3 = max3(mx3, v[e + 6], v[e + 7]);
-      }
-      mx0 = max3(mx0, v[BN - 4], v[BN - 3]);
-      mx1 = max3(mx1, v[BN - 2], v[BN - 1]);
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * c_j;
+      const float mx = mx_raw * c_j;
       const float m_new = fmaxf(m_run, mx);
       float alpha = 1.f;
       const bool resc = (m_new - m_run) > kRescaleThreshold;
@@ -464,6 +479,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       float ls = (acc0.x + acc0.y) + (acc1.x + acc1.y);
+      if (n_left_out != 0.f) ls = fmaf(-n_left_out, ex2_approx(neg_m), ls);   // zero-logit keys left out
       if constexpr (FP8) ls *= ex2_approx(-bias);
       l_run += ls;
       tc_fence_before();

@@ -343,6 +343,8 @@ jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt,
     g.idx = idx;
     g.k_out = ws + L.kr;
     g.v_out = ws + L.vr;
+    g.k8 = ws + L.k8;
+    g.v8 = ws + L.v8;
     g.status = status_ptr();
     if (jattn::launch_repair_gather(g, cs) != cudaSuccess) return JATTN_ERR_CUDA;
   }

@@ -38,6 +38,8 @@ struct GatherParams {
   const int32_t* idx;           // [B*H][n] token indices
   void* k_out;                  // fp16 [B*H][n][d], rotated (and normalised) keys
   void* v_out;                  // fp16 [B*H][n][d]
+  uint8_t* k8;                  // e4m3 [B*H][S][d] keys / values of the FP8 pass: the repaired
+  uint8_t* v8;                  //   tokens' rows are set to code 0 (logit exactly 0, value 0)
   uint32_t* status;
 };
 

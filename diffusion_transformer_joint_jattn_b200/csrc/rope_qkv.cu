@@ -415,6 +415,19 @@ __global__ void __launch_bounds__(256) repair_gather_kernel(const GatherParams p
     kw[j] = pack_f16(k[2 * j], k[2 * j + 1]);
     vw[j] = pack_f16(v[2 * j], v[2 * j + 1]);
   }
+  // The FP8 pass sees this token's key and value as zero codes: its logit is
+  // exactly 0 and it adds nothing to O (the pass removes its probability
+  // from the row sum, see the key mask in the forward kernel).
+  {
+    const size_t off8 = (static_cast<size_t>(bh) * p.S + t) * D + c0;
+    if constexpr (CPL == 4) {
+      *reinterpret_cast<uint32_t*>(p.k8 + off8) = 0u;
+      *reinterpret_cast<uint32_t*>(p.v8 + off8) = 0u;
+    } else {
+      *reinterpret_cast<uint16_t*>(p.k8 + off8) = 0u;
+      *reinterpret_cast<uint16_t*>(p.v8 + off8) = 0u;
+    }
+  }
   const size_t off = (static_cast<size_t>(bh) * p.n + r) * D + c0;
   uint16_t* ko = static_cast<uint16_t*>(p.k_out) + off;
   uint16_t* vo = static_cast<uint16_t*>(p.v_out) + off;
