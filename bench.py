@@ -379,24 +379,40 @@ def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
     """Run the FP64 oracle on `heads` (b, h) pairs x `rows_per_head` query
     rows of workload w.  Returns (seconds, flops)."""
     import oracle
+    from threadpoolctl import threadpool_limits
     sub = w.with_batch_heads(B=1, H=heads)
     inp = W.make_inputs(sub, seed)
     rows = W.sample_rows(sub, rows_per_head, seed)
-    workers = max(1, (os.cpu_count() or 2) // 2)
-    t = time.perf_counter()
-    oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], sub.split, sub.theta,
-                           rows=rows, workers=workers)
-    dt = time.perf_counter() - t
+    # One worker thread per host core, each with a single-threaded BLAS, so
+    # the threads used are exactly `workers`.
+    workers = max(1, os.cpu_count() or 1)
+    with threadpool_limits(1):
+        t = time.perf_counter()
+        oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], sub.split, sub.theta,
+                               rows=rows, workers=workers)
+        dt = time.perf_counter() - t
     return dt, 4 * heads * rows.shape[-1] * w.S * w.d, workers
+
+
+def host_workers() -> int:
+    """Worker threads of the oracle timing: one per host core."""
+    return max(1, os.cpu_count() or 1)
+
+
+def round_heads(w, n: float, workers: int) -> int:
+    """A head count for a sample: the oracle runs one head per worker thread,
+    so a multiple of the worker count (at most B*H) keeps every core busy."""
+    return int(max(1, min(w.B * w.H, -(-int(math.ceil(n)) // workers) * workers)))
 
 
 def cpu_baseline(w, target_s: float = 12.0):
     # Calibrate on a small sample, then size the sample for ~target_s seconds.
     # The small sample carries per-head fixed costs (rotating every key), so
     # the first estimate runs short: rescale once more from the real run.
-    dt, fl, _ = oracle_sample(w, 128, 2)
+    workers = host_workers()
+    heads = round_heads(w, 1, workers)
+    dt, fl, _ = oracle_sample(w, 128, heads)
     rate = fl / dt
-    heads = 8
     rows = int(max(128, min(w.S, target_s * rate / (4 * heads * w.S * w.d))))
     dt, fl, workers = oracle_sample(w, rows, heads)
     for _ in range(3):
@@ -406,9 +422,9 @@ def cpu_baseline(w, target_s: float = 12.0):
         if rows < w.S:
             rows = int(min(w.S, rows * grow))
         else:
-            heads = int(min(w.B * w.H, max(heads + 1, heads * grow)))
+            heads = round_heads(w, max(heads + 1, heads * grow), workers)
         dt, fl, workers = oracle_sample(w, rows, heads)
-    return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": os.cpu_count(), "threads": workers,
+    return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": workers, "blas_threads_per_worker": 1,
             "kind": "oracle",
             "sample": f"{heads} heads x {rows} sampled query rows of {w.name} (S={w.S}, d={w.d}), "
                       f"FP64 numpy oracle incl. RoPE, {dt:.1f} s"}
@@ -419,14 +435,15 @@ def run_reference(args, rank, world):
         return
     w = W.BY_NAME[args.workload]
     flops = 4 * w.B * w.H * w.S * w.S * w.d
-    dt, fl, workers = oracle_sample(w, 128, 2)
+    heads = round_heads(w, 1, host_workers())
+    dt, fl, workers = oracle_sample(w, 128, heads)
     rate = fl / dt
     steps_budget_s = 150.0
     per_step_s = max(1.0, steps_budget_s / max(1, args.steps + args.warmup))
-    rows = int(max(32, min(w.S, per_step_s * rate / (4 * 2 * w.S * w.d))))
+    rows = int(max(32, min(w.S, per_step_s * rate / (4 * heads * w.S * w.d))))
     times = []
     for i in range(args.warmup + args.steps):
-        dt, fl, workers = oracle_sample(w, rows, 2, seed=i)
+        dt, fl, workers = oracle_sample(w, rows, heads, seed=i)
         if i >= args.warmup:
             times.append(dt)
     sec = float(np.mean(times))
@@ -436,10 +453,10 @@ def run_reference(args, rank, world):
             "warmup": args.warmup, "ms_per_step": round(ms_full, 1), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "d": w.d,
-                       "note": "each step = FP64 oracle on 2 heads x %d sampled rows; ms_per_step extrapolated "
-                               "to the full call from the sampled rate" % rows},
-            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": os.cpu_count(), "threads": workers,
-                             "kind": "oracle", "sample": f"2 heads x {rows} query rows per step"},
+                       "note": "each step = FP64 oracle on %d heads x %d sampled rows; ms_per_step extrapolated "
+                               "to the full call from the sampled rate" % (heads, rows)},
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": workers, "blas_threads_per_worker": 1,
+                             "kind": "oracle", "sample": f"{heads} heads x {rows} query rows per step"},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
