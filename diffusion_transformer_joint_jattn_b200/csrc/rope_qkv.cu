@@ -17,7 +17,8 @@
 // entry and walks all 3*H (Q/K/V, head) tiles of it, so each (token, pair)
 // cos/sin is computed once per CTA and lives in registers; loads and stores
 // are 16-byte vectors, coalesced along d; the next tile's loads are issued
-// before the current tile is processed.  For e4m3 output the tile's amax is
+// before the current tile is processed, and the one after it is prefetched
+// into L2.  For e4m3 output the tile's amax is
 // reduced across the CTA before its codes are written, so every input byte is
 // read exactly once.  The RMSNorm's sum of squares is a shuffle reduction over
 // the D/8 consecutive lanes that hold one row; its weights are staged in
@@ -155,7 +156,20 @@ rope_qkv_kernel(const RopeParams p) {
     for (int i = 0; i < kTokPerThread; ++i)
       buf[i] = valid[i] ? __ldg(reinterpret_cast<const uint4*>(src[i] + off)) : make_uint4(0, 0, 0, 0);
   };
+  // The tile after the one held in registers is asked into L2 ahead of its
+  // load: one 512-thread CTA per SM keeps too few bytes in flight with the
+  // register prefetch alone.  One lane per 128-byte line issues it.
+  auto prefetch_item_l2 = [&](int item) {
+    const int which = item / H, h = item % H;
+    const size_t off = static_cast<size_t>(which * H + h) * D;
+    if ((cg & 7) == 0) {
+#pragma unroll
+      for (int i = 0; i < kTokPerThread; ++i)
+        if (valid[i]) asm volatile("prefetch.global.L2 [%0];" ::"l"(src[i] + off));
+    }
+  };
   load_item(0, nxt);
+  if (items > 1) prefetch_item_l2(1);
   bool range_hit = false;
 
   for (int item = 0; item < items; ++item) {
@@ -163,6 +177,7 @@ rope_qkv_kernel(const RopeParams p) {
 #pragma unroll
     for (int i = 0; i < kTokPerThread; ++i) cur[i] = nxt[i];
     if (item + 1 < items) load_item(item + 1, nxt);
+    if (item + 2 < items) prefetch_item_l2(item + 2);
     const int which = item / H, h = item % H;
 
     float x[kTokPerThread][8];
