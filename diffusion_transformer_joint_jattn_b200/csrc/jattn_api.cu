@@ -164,7 +164,7 @@ RepairLayout repair_layout(const jattn_shape* shape, int n) {
   L.v8 = seg(BH * S * d);
   L.scales = seg(3 * BH * nb * 4);
   L.q16 = seg(BH * S * d * 2);
-  L.score = seg(BH * S * 4);
+  L.score = seg(2 * BH * S * 4);
   L.idx = seg(BH * n * 4);
   L.kmask = seg(BH * nb * 16);
   L.kr = seg(BH * n * d * 2);

@@ -21,7 +21,7 @@ struct RopeParams {
   const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
   float eps;                    // RMSNorm epsilon
   void* q16;                    // e4m3 output with token repair: also fp16 Q [B, H, S, d], else null
-  float* score;                 // with token repair: |k|^2 + |v|^2 per token [B, H, S], else null
+  float* score;                 // with token repair: [2][B, H, S], |k|^2 then |v|^2 per token, else null
   uint32_t* status;
 };
 
@@ -44,9 +44,11 @@ struct GatherParams {
 };
 
 cudaError_t launch_repair_gather(const GatherParams& p, cudaStream_t st);
-// Per (b, h): the n largest scores (ties to the lower index) -> idx [B*H][n]
-// in index order, and the key mask [B*H][n_kv][4] words with their bits set.
-cudaError_t launch_repair_select(const float* score, int BH, int S, int n, int n_kv, int32_t* idx,
+// Per (b, h): the n largest scores |k|^2 + |v|^2 (ties to the lower index)
+// -> idx [B*H][n] in index order, and the key mask [B*H][n_kv][4] words with
+// their bits set.  score holds the [2][B*H][S] K and V planes; the K plane is
+// overwritten with the sums.
+cudaError_t launch_repair_select(float* score, int BH, int S, int n, int n_kv, int32_t* idx,
                                  uint32_t* kmask, cudaStream_t st);
 
 struct QuantParams {

@@ -54,17 +54,23 @@ __device__ uint32_t block_exclusive_scan(uint32_t x, uint32_t* warp_sums, uint32
   return before + incl - x;
 }
 
-__global__ void __launch_bounds__(kSelThreads) repair_select_kernel(const float* __restrict__ score, int S, int n,
-                                                                    int n_kv, int32_t* __restrict__ idx,
+// score: [2][B*H][S], the |k|^2 plane then the |v|^2 plane; the K plane is
+// overwritten with the sums.
+__global__ void __launch_bounds__(kSelThreads) repair_select_kernel(float* score, int S, int n, int n_kv,
+                                                                    int32_t* __restrict__ idx,
                                                                     uint32_t* __restrict__ kmask) {
   __shared__ uint32_t hist[256];
   __shared__ uint32_t warp_sums[32];
   __shared__ uint32_t s_prefix, s_rank;
   const int tid = threadIdx.x;
   const size_t bh = blockIdx.x;
-  const uint32_t* sc = reinterpret_cast<const uint32_t*>(score) + bh * S;
+  float* sk = score + bh * S;
+  const float* sv = score + static_cast<size_t>(gridDim.x) * S + bh * S;
+  for (int i = tid; i < S; i += kSelThreads) sk[i] = sk[i] + sv[i];
   uint32_t* mask = kmask + bh * static_cast<size_t>(n_kv) * 4;
   for (int w = tid; w < n_kv * 4; w += kSelThreads) mask[w] = 0u;
+  __syncthreads();
+  const uint32_t* sc = reinterpret_cast<const uint32_t*>(sk);
 
   // Radix select: after the pass for bits [shift, shift+8), `prefix` holds the
   // top bits of T and `rank` the position (1-based, from the top) of T among
@@ -127,7 +133,7 @@ __global__ void __launch_bounds__(kSelThreads) repair_select_kernel(const float*
 
 }  // namespace
 
-cudaError_t launch_repair_select(const float* score, int BH, int S, int n, int n_kv, int32_t* idx,
+cudaError_t launch_repair_select(float* score, int BH, int S, int n, int n_kv, int32_t* idx,
                                  uint32_t* kmask, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   repair_select_kernel<<<BH, kSelThreads, 0, st>>>(score, S, n, n_kv, idx, kmask);

@@ -237,10 +237,10 @@ rope_qkv_kernel(const RopeParams p) {
 #pragma unroll
           for (int o = CG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
           if (cg == 0 && valid[i]) {
-            // K comes before V in the item order and the same lane owns the
-            // token in both, so the V pass reads back its own K term.
-            float* sc = p.score + row0 + tok[i];
-            *sc = which == 1 ? ss : *sc + ss;
+            // K and V terms go to separate planes (the selection adds them):
+            // no pass waits on a read of what an earlier one wrote.
+            const size_t plane = which == 2 ? static_cast<size_t>(p.B) * H * S : 0;
+            p.score[plane + row0 + tok[i]] = ss;
           }
         }
       }
