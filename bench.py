@@ -30,11 +30,13 @@ sys.path.insert(0, ROOT)
 from diffusion_transformer_joint_jattn_b200 import workloads as W  # noqa: E402
 
 WORKLOAD = "t2i_2048_base"
-# DRAM bytes per launch of the forward kernel on t2i_2048_base: the ncu
-# capture of the same kernel on t2i_1024_base (profiles/attn_fwd_t2i_1024_base.md,
-# dram__bytes_read.sum + dram__bytes_write.sum = 207.44 MB) scaled by the token
-# count 16896 / 4608 (the traffic is Q, K, V and O once each, linear in tokens).
-FWD_TRAFFIC_BYTES = 206.96e6 * 16896 / 4608
+# DRAM bytes per launch of the forward kernels on t2i_2048_base: the ncu
+# captures of the same kernels on t2i_1024_base (dram__bytes_read.sum +
+# dram__bytes_write.sum: 205.21 MB with fp16 operands, 109.19 MB with e4m3
+# operands) scaled by the token count 16896 / 4608 (the traffic is Q, K, V
+# and O once each, linear in tokens).
+FWD_TRAFFIC_BYTES = 205.21e6 * 16896 / 4608
+FWD_FP8_TRAFFIC_BYTES = 109.19e6 * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 
@@ -231,7 +233,10 @@ def run_ours(args, rank, world, local):
                             "peak": round(2 * peaks["bf16_tflops_sustained"], 1), "unit": "TFLOP/s",
                             "frac": round(flops / fwd8 / 1e9 / (2 * peaks["bf16_tflops_sustained"]), 4),
                             "peak_note": f"fp8 = 2 x {peak_src} bf16 sustained (nominal fp8/bf16 ratio)",
-                            "frac_of_nominal_4500": round(flops / fwd8 / 1e9 / 4500.0, 4), "traffic": None}}
+                            "frac_of_nominal_4500": round(flops / fwd8 / 1e9 / 4500.0, 4),
+                            "traffic": round(FWD_FP8_TRAFFIC_BYTES) if args.workload == WORKLOAD else None,
+                            "traffic_note": "ncu capture on t2i_1024_base scaled by tokens (see profiles/)",
+                            "kernel": "attn_fwd_kernel<128, e4m3 operands>"}}
 
     extras = {}
     if not args.no_extras:
