@@ -6,10 +6,14 @@ e4m3 pair for the FP8 path).  TFLOPS = 4 * B * H * S^2 * d / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Under torchrun each rank runs the same workload on its own GPU with its own
-seed (weak scaling, no data-path collective); the step time is the max over
-ranks.  ``--impl reference`` times the FP64 oracle on the host cores instead
-(rank 0 only), on bounded samples of the same workload.
+With one GPU the whole batch runs on it.  Under torchrun (N > 1) the batch is
+partitioned the way the multi-GPU mode of the page does it: the two
+classifier-free-guidance branches (batch entries) on separate rank groups,
+each branch's sequence over the ranks of its group with Ulysses sequence
+parallelism (two NCCL all-to-alls around the unchanged device path).  The
+total work is fixed (strong scaling); the step time is the max over ranks.
+``--impl reference`` times the FP64 oracle on the host cores instead (rank 0
+only), on bounded samples of the same workload.
 """
 from __future__ import annotations
 
@@ -39,9 +43,12 @@ FWD_TRAFFIC_BYTES = 205.21e6 * 16896 / 4608
 FWD_FP8_TRAFFIC_BYTES = 109.19e6 * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
+# Per-sample time of the oracle on the host cores (both CPU legs use the same
+# sample shape, so their rates agree).
+ORACLE_SAMPLE_S = 6.0
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -52,9 +59,9 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
-                    help="skip the FP8-with-repair and query/key-norm prologue measurements")
+                    help="skip the FP8-with-repair, query/key-norm prologue and other-workload measurements")
     ap.add_argument("--rho", type=float, default=0.005, help="token-repair budget of the FP8-with-repair block")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def dist_env():
@@ -74,15 +81,10 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
-def whole_job_tflops(world: int, flops_per_rank: int, ms_per_step: float) -> float:
-    """Aggregate throughput: every rank processes its own batch (weak
-    scaling), the step takes the slowest rank's time."""
-    return world * flops_per_rank / ms_per_step / 1e9
-
-
-def rank_seed(rank: int) -> int:
-    """Each rank draws its own synthetic batch."""
-    return rank
+def whole_job_tflops(flops_total: int, ms_per_step: float) -> float:
+    """Aggregate throughput: the whole batch's FLOPs over the slowest rank's
+    step time."""
+    return flops_total / ms_per_step / 1e9
 
 
 def load_peaks():
@@ -142,204 +144,23 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def run_ours(args, rank, world, local):
-    from diffusion_transformer_joint_jattn_b200 import jattn
-    import torch.distributed as dist
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
-    w = W.BY_NAME[args.workload]
-    B, H, S, d = w.B, w.H, w.S, w.d
-    flops = 4 * B * H * S * S * d
-    inp = W.make_inputs(w, seed=rank_seed(rank))
-    dinp = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
-    stream = torch.cuda.current_stream()
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_ranks(x: float) -> float:
-        return max_over_ranks(x, world, dev)
-
-    spread = {}                                           # per path: median / min of the timed forwards
-
-    def measure(path: str, steps: int, warmup: int):
-        """Time `steps` whole-path steps; events around each kernel."""
-        if path == "bf16":
-            q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
-            bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
-        else:
-            q = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=dev)
-            bufs = (q, torch.empty_like(q), torch.empty_like(q),
-                    torch.empty(3, B, H, jattn.n_blocks(S), dtype=torch.float32, device=dev))
-        o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
-
-        def step(ev=None):
-            if ev is not None:
-                ev[0].record(stream)
-            if path == "bf16":
-                jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
-                               "fp16", out=bufs, stream=stream)
-                if ev is not None:
-                    ev[1].record(stream)
-                jattn.fwd_bf16(bufs[0], bufs[1], bufs[2], o=o, stream=stream)
-            else:
-                jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
-                               "e4m3", out=bufs, stream=stream)
-                if ev is not None:
-                    ev[1].record(stream)
-                jattn.fwd_fp8(bufs[0], bufs[1], bufs[2], bufs[3], o=o, stream=stream)
-            if ev is not None:
-                ev[2].record(stream)
-
-        for _ in range(warmup):
-            step()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
-        barrier()
-        torch.cuda.synchronize()
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(steps):
-            step(evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        total_ms = t0.elapsed_time(t1)
-        pro = float(np.mean([e[0].elapsed_time(e[1]) for e in evs]))
-        fwd_all = [e[1].elapsed_time(e[2]) for e in evs]
-        fwd = float(np.mean(fwd_all))
-        code, bits = jattn.device_status(clear=True)
-        if code != jattn.OK:
-            raise RuntimeError(f"device status {code} bits {bits} after the {path} run")
-        spread[path] = {"fwd_ms_median": round(max_ranks(float(np.median(fwd_all))), 4),
-                        "fwd_ms_min": round(max_ranks(float(np.min(fwd_all))), 4)}
-        return max_ranks(total_ms / steps), max_ranks(pro), max_ranks(fwd)
-
-    peaks, peak_src = load_peaks()
-    sampler = ClockSampler(local)
-    sampler.start()
-    ms, pro_ms, fwd_ms = measure("bf16", args.steps, args.warmup)
-    clocks = sampler.stop()
-    fp8 = None
-    if not args.no_fp8:
-        ms8, pro8, fwd8 = measure("fp8", args.steps, args.warmup)
-        fp8 = {"value": round(whole_job_tflops(world, flops, ms8), 2), "unit": UNIT, "ms_per_step": round(ms8, 4),
-               "prologue_ms": round(pro8, 4), "fwd_ms": round(fwd8, 4), **spread["fp8"],
-               "roofline": {"bound": "tensor", "achieved": round(flops / fwd8 / 1e9, 2),
-                            "peak": round(2 * peaks["bf16_tflops_sustained"], 1), "unit": "TFLOP/s",
-                            "frac": round(flops / fwd8 / 1e9 / (2 * peaks["bf16_tflops_sustained"]), 4),
-                            "peak_note": f"fp8 = 2 x {peak_src} bf16 sustained (nominal fp8/bf16 ratio)",
-                            "frac_of_nominal_4500": round(flops / fwd8 / 1e9 / 4500.0, 4),
-                            "traffic": round(FWD_FP8_TRAFFIC_BYTES) if args.workload == WORKLOAD else None,
-                            "traffic_note": "ncu capture on t2i_1024_base scaled by tokens (see profiles/)",
-                            "kernel": "attn_fwd_kernel<128, e4m3 operands>"}}
-
-    extras = {}
-    if not args.no_extras:
-        extras = measure_extras(jattn, w, dinp, dev, stream, args, flops, world, max_ranks, barrier,
-                                ms8 if fp8 is not None else None)
-
-    e2e = None
-    if not args.no_e2e:
-        e2e = measure_e2e(jattn, w, inp, dev, stream, min(args.steps, 10), 2, flops, world, max_ranks, barrier)
-
+def tensor_roofline(flops: int, fwd_ms: float, peaks, peak_src: str, fp8: bool, traffic, kernel: str):
+    """Roofline of one forward launch: algorithmic FLOPs / its CUDA-event
+    duration against the measured burst cuBLAS bf16 rate (the forward is a
+    few-millisecond kernel timed in a sub-second region); FP8 against twice
+    that (the nominal fp8 / bf16 ratio)."""
+    mult = 2.0 if fp8 else 1.0
     achieved = flops / fwd_ms / 1e9
-    peak = peaks["bf16_tflops_sustained"]
-    line = {
-        "metric": METRIC, "value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT, "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
-        "config": {"workload": w.name, "B": B, "H": H, "S": S, "S_txt": w.S_txt, "S_img": w.S_img,
-                   "S_ref": w.S_ref, "d": d, "rope_split": list(w.split), "theta": w.theta,
-                   "path": "bf16 in/out, fp16 MMA operands, fp32 accumulate",
-                   "l2": "inputs larger than L2 (623 MB qkv streams, 622 MB laid-out q/k/v)",
-                   "parallelism": f"replicas x{world}"},
-        "prologue_ms": round(pro_ms, 4), "fwd_ms": round(fwd_ms, 4), **spread["bf16"],
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4),
-                     "peak_note": f"{peak_src} cuBLAS bf16 sustained (MEASURED_PEAKS.json bf16_tflops_sustained)",
-                     "frac_of_burst": round(achieved / peaks["bf16_tflops"], 4),
-                     "frac_of_nominal_2250": round(achieved / 2250.0, 4),
-                     "traffic": round(FWD_TRAFFIC_BYTES) if args.workload == WORKLOAD else None,
-                     "traffic_note": "ncu capture on t2i_1024_base scaled by tokens (see profiles/)",
-                     "kernel": "attn_fwd_kernel<128, fp16 operands>"},
-        "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / pro_ms / 1e6, 1),
-                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                              "frac": round(prologue_bytes(w, 2) / pro_ms / 1e6 / peaks["hbm_gbs"], 4)},
-        "gpu_launches": 2 * args.steps,
-        "clocks": clocks,
-    }
-    if fp8 is not None:
-        line["fp8"] = fp8
-    line.update(extras)
-    if e2e is not None:
-        line["e2e"] = e2e
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, target_s=12.0)
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
-
-
-def _timed(fn, stream, steps, warmup, barrier, max_ranks):
-    for _ in range(warmup):
-        fn()
-    barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        fn()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    return max_ranks(t0.elapsed_time(t1) / steps)
-
-
-def measure_extras(jattn, w, dinp, dev, stream, args, flops, world, max_ranks, barrier, ms_fp8):
-    """The next-row paths, timed the same way (device events around the
-    call, inputs resident, workspace allocated beforehand):
-    * FP8 attention with token repair (the whole call: prologue, selection,
-      gather, masked FP8 pass, merged fp16 pass);
-    * the prologue with the query/key RMSNorm fused in, against the same
-      prologue without it."""
-    B, H, S, d = w.B, w.H, w.S, w.d
-    out = {}
-    rho = args.rho
-    n = jattn.repair_count(B, H, w.S_txt, w.S_img, w.S_ref, d, rho)
-    ws = torch.empty(jattn.repair_workspace_bytes(B, H, w.S_txt, w.S_img, w.S_ref, d, rho), dtype=torch.uint8,
-                     device=dev)
-    o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
-    ms = _timed(lambda: jattn.fwd_fp8_repair(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"],
-                                             w.split, w.theta, rho=rho, workspace=ws, o=o, stream=stream),
-                stream, args.steps, args.warmup, barrier, max_ranks)
-    code, bits = jattn.device_status(clear=True)
-    if code != jattn.OK:
-        raise RuntimeError(f"device status {code} bits {bits} after the FP8-with-repair run")
-    out["fp8_repair"] = {"value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT,
-                         "ms_per_step": round(ms, 4), "rho": rho, "repaired_per_head": n,
-                         "workspace_bytes": ws.numel(), "gpu_launches_per_step": 5 if n else 2,
-                         "overhead_vs_fp8": None if ms_fp8 is None else round(ms / ms_fp8 - 1, 4)}
-    del ws, o
-    q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
-    bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
-    nw = W.norm_weights(d, 0).to(dev)
-    res = {}
-    for name, norm in (("plain", None), ("qk_norm", nw)):
-        res[name] = _timed(lambda: jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"],
-                                                  w.split, w.theta, "fp16", out=bufs, stream=stream, norm_w=norm),
-                           stream, args.steps, args.warmup, barrier, max_ranks)
-    nbytes = prologue_bytes(w, 2)
-    out["prologue_qk_norm"] = {"ms": round(res["qk_norm"], 4), "ms_without_norm": round(res["plain"], 4),
-                               "achieved_GBps": round(nbytes / res["qk_norm"] / 1e6, 1),
-                               "note": "fp16 output; back-to-back calls (no flush between them)"}
-    return out
+    peak = mult * peaks["bf16_tflops"]
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4),
+            "peak_note": (f"{'2 x ' if fp8 else ''}{peak_src} cuBLAS bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                          + (", nominal fp8 / bf16 ratio" if fp8 else "")),
+            "frac_of_sustained": round(achieved / (mult * peaks["bf16_tflops_sustained"]), 4),
+            "frac_of_nominal": round(achieved / (4500.0 if fp8 else 2250.0), 4),
+            "traffic": None if traffic is None else round(traffic),
+            "traffic_note": "ncu capture on t2i_1024_base scaled by tokens (see profiles/)",
+            "kernel": kernel}
 
 
 def prologue_bytes(w, out_bytes: int) -> int:
@@ -349,40 +170,306 @@ def prologue_bytes(w, out_bytes: int) -> int:
     return n * 2 + n * out_bytes
 
 
-def measure_e2e(jattn, w, inp, dev, stream, steps, warmup, flops, world, max_over_ranks, barrier):
+class Ctx:
+    """What the timing helpers share: device, stream, world size, barrier."""
+
+    def __init__(self, dev, world):
+        self.dev = dev
+        self.world = world
+        self.stream = torch.cuda.current_stream()
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max_ranks(self, x: float) -> float:
+        return max_over_ranks(x, self.world, self.dev)
+
+
+def time_calls(ctx: Ctx, fn, steps: int, warmup: int, marks: int = 0):
+    """Run ``fn(ev)`` warmup times untimed, then ``steps`` times between two
+    events on the stream; ``fn`` records ``marks`` inner events (``ev`` list)
+    around the kernels it launches.  Returns (ms per call, per-call inner
+    intervals [steps][marks-1] in ms), max over ranks."""
+    for _ in range(warmup):
+        fn(None)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(marks)] for _ in range(steps)]
+    ctx.barrier()
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(ctx.stream)
+    for i in range(steps):
+        fn(evs[i] if marks else None)
+    t1.record(ctx.stream)
+    torch.cuda.synchronize()
+    ctx.barrier()
+    inner = [[e[k].elapsed_time(e[k + 1]) for k in range(marks - 1)] for e in evs] if marks else []
+    return ctx.max_ranks(t0.elapsed_time(t1) / steps), inner
+
+
+def path_step(jattn, w, dinp, path: str, dev, stream):
+    """Buffers and a step function for one whole-path step (prologue +
+    forward) of workload w; the step records 3 events when given them."""
+    B, H, S, d = w.B, w.H, w.S, w.d
+    if path == "bf16":
+        q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
+        bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
+    else:
+        q = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=dev)
+        bufs = (q, torch.empty_like(q), torch.empty_like(q),
+                torch.empty(3, B, H, jattn.n_blocks(S), dtype=torch.float32, device=dev))
+    o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
+
+    def step(ev):
+        if ev is not None:
+            ev[0].record(stream)
+        jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                       "fp16" if path == "bf16" else "e4m3", out=bufs, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        if path == "bf16":
+            jattn.fwd_bf16(bufs[0], bufs[1], bufs[2], o=o, stream=stream)
+        else:
+            jattn.fwd_fp8(bufs[0], bufs[1], bufs[2], bufs[3], o=o, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    return step
+
+
+def measure_path(jattn, ctx: Ctx, w, dinp, path: str, steps: int, warmup: int):
+    """Whole-path steps of one workload: (ms per step, mean prologue ms, mean
+    forward ms, median forward ms, min forward ms), max over ranks."""
+    step = path_step(jattn, w, dinp, path, ctx.dev, ctx.stream)
+    ms, inner = time_calls(ctx, step, steps, warmup, marks=3)
+    code, bits = jattn.device_status(clear=True)
+    if code != jattn.OK:
+        raise RuntimeError(f"device status {code} bits {bits} after the {path} run of {w.name}")
+    pro = [x[0] for x in inner]
+    fwd = [x[1] for x in inner]
+    return (ms, ctx.max_ranks(float(np.mean(pro))), ctx.max_ranks(float(np.mean(fwd))),
+            ctx.max_ranks(float(np.median(fwd))), ctx.max_ranks(float(np.min(fwd))))
+
+
+def run_ours(args, rank, world, local):
+    if world > 1:
+        return run_partition(args, rank, world, local)
+    from diffusion_transformer_joint_jattn_b200 import jattn
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ctx = Ctx(dev, world)
+    w = W.BY_NAME[args.workload]
+    B, H, S, d = w.B, w.H, w.S, w.d
+    flops = w.flops
+    inp = W.make_inputs(w, seed=0)
+    dinp = {k: (None if v is None else v.to(dev)) for k, v in inp.items()}
+    peaks, peak_src = load_peaks()
+    full = args.workload == WORKLOAD
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms, pro_ms, fwd_ms, fwd_med, fwd_min = measure_path(jattn, ctx, w, dinp, "bf16", args.steps, args.warmup)
+    clocks = sampler.stop()
+    fp8 = None
+    if not args.no_fp8:
+        ms8, pro8, fwd8, fwd8_med, fwd8_min = measure_path(jattn, ctx, w, dinp, "fp8", args.steps, args.warmup)
+        fp8 = {"value": round(whole_job_tflops(flops, ms8), 2), "unit": UNIT, "ms_per_step": round(ms8, 4),
+               "prologue_ms": round(pro8, 4), "fwd_ms": round(fwd8, 4), "fwd_ms_median": round(fwd8_med, 4),
+               "fwd_ms_min": round(fwd8_min, 4),
+               "roofline": tensor_roofline(flops, fwd8, peaks, peak_src, True,
+                                           FWD_FP8_TRAFFIC_BYTES if full else None,
+                                           "attn_fwd_kernel<128, e4m3 operands>")}
+
+    extras = {}
+    if not args.no_extras:
+        extras = measure_extras(jattn, ctx, w, dinp, args, flops, ms8 if fp8 is not None else None)
+        extras["workloads"] = measure_other_workloads(jattn, ctx, args)
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(jattn, ctx, w, inp, min(args.steps, 10), 2, flops)
+
+    line = {
+        "metric": METRIC, "value": round(whole_job_tflops(flops, ms), 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "H": H, "S": S, "S_txt": w.S_txt, "S_img": w.S_img,
+                   "S_ref": w.S_ref, "d": d, "rope_split": list(w.split), "theta": w.theta,
+                   "path": "bf16 in/out, fp16 MMA operands, fp32 accumulate (jattn_rope_qkv + jattn_fwd_bf16)",
+                   "l2": "inputs larger than L2 (623 MB qkv streams, 622 MB laid-out q/k/v)",
+                   "parallelism": "single GPU"},
+        "prologue_ms": round(pro_ms, 4), "fwd_ms": round(fwd_ms, 4), "fwd_ms_median": round(fwd_med, 4),
+        "fwd_ms_min": round(fwd_min, 4),
+        "roofline": tensor_roofline(flops, fwd_ms, peaks, peak_src, False, FWD_TRAFFIC_BYTES if full else None,
+                                    "attn_fwd_kernel<128, fp16 operands>"),
+        "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / pro_ms / 1e6, 1),
+                              "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                              "frac": round(prologue_bytes(w, 2) / pro_ms / 1e6 / peaks["hbm_gbs"], 4),
+                              "peak_note": f"{peak_src} HBM copy bandwidth"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if fp8 is not None:
+        line["fp8"] = fp8
+    line.update(extras)
+    if e2e is not None:
+        line["e2e"] = e2e
+    if rank == 0 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops, ms_fp8):
+    """The next-row paths on the headline workload, timed the same way
+    (device events around the call, inputs resident, workspace allocated
+    beforehand):
+    * FP8 attention with token repair (the whole call: prologue, selection,
+      gather, masked FP8 pass, merged fp16 pass);
+    * the prologue with the query/key RMSNorm fused in, against the same
+      prologue without it."""
+    out = {"fp8_repair": measure_repair(jattn, ctx, w, dinp, args.rho, args.steps, args.warmup, ms_fp8)}
+    B, H, S, d = w.B, w.H, w.S, w.d
+    q = torch.empty(B, H, S, d, dtype=torch.float16, device=ctx.dev)
+    bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
+    nw = W.norm_weights(d, 0).to(ctx.dev)
+    res = {}
+    for name, norm in (("plain", None), ("qk_norm", nw)):
+        res[name], _ = time_calls(
+            ctx, lambda ev: jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split,
+                                           w.theta, "fp16", out=bufs, stream=ctx.stream, norm_w=norm),
+            args.steps, args.warmup)
+    nbytes = prologue_bytes(w, 2)
+    out["prologue_qk_norm"] = {"ms": round(res["qk_norm"], 4), "ms_without_norm": round(res["plain"], 4),
+                               "achieved_GBps": round(nbytes / res["qk_norm"] / 1e6, 1),
+                               "note": "fp16 output; back-to-back calls (no flush between them)"}
+    return out
+
+
+def measure_repair(jattn, ctx: Ctx, w, dinp, rho, steps, warmup, ms_fp8):
+    B, H, S, d = w.B, w.H, w.S, w.d
+    n = jattn.repair_count(B, H, w.S_txt, w.S_img, w.S_ref, d, rho)
+    ws = torch.empty(jattn.repair_workspace_bytes(B, H, w.S_txt, w.S_img, w.S_ref, d, rho), dtype=torch.uint8,
+                     device=ctx.dev)
+    o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=ctx.dev)
+    ms, _ = time_calls(ctx, lambda ev: jattn.fwd_fp8_repair(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"],
+                                                            dinp["pos"], w.split, w.theta, rho=rho, workspace=ws,
+                                                            o=o, stream=ctx.stream), steps, warmup)
+    code, bits = jattn.device_status(clear=True)
+    if code != jattn.OK:
+        raise RuntimeError(f"device status {code} bits {bits} after the FP8-with-repair run")
+    return {"value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
+            "rho": rho, "repaired_per_head": n, "workspace_bytes": ws.numel(), "gpu_launches_per_step": 5 if n else 2,
+            "overhead_vs_fp8": None if ms_fp8 is None else round(ms / ms_fp8 - 1, 4)}
+
+
+def measure_other_workloads(jattn, ctx: Ctx, args):
+    """Throughput on the other 2048x2048 workloads: the distilled T2I (B = 1,
+    FP8 plain and with token repair) and the I2I with one reference image
+    (S = 33280, BF16 and FP8).  Fewer steps: each is a few-second run."""
+    peaks, peak_src = load_peaks()
+    steps, warmup = max(3, min(args.steps, 10)), 3
+    out = {}
+    for name, paths in (("t2i_2048_distilled", ("fp8",)), ("i2i_2048_base", ("bf16", "fp8"))):
+        w = W.BY_NAME[name]
+        dinp = {k: (None if v is None else v.to(ctx.dev)) for k, v in W.make_inputs(w, 0).items()}
+        res = {"B": w.B, "S": w.S, "flops_per_call": w.flops}
+        ms_fp8 = None
+        for path in paths:
+            ms, pro, fwd, _, _ = measure_path(jattn, ctx, w, dinp, path, steps, warmup)
+            if path == "fp8":
+                ms_fp8 = ms
+            res[path] = {"value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
+                         "prologue_ms": round(pro, 4), "fwd_ms": round(fwd, 4),
+                         "roofline": tensor_roofline(w.flops, fwd, peaks, peak_src, path == "fp8", None,
+                                                     f"attn_fwd_kernel<128, {'e4m3' if path == 'fp8' else 'fp16'} "
+                                                     "operands>")}
+        if name == "t2i_2048_distilled":
+            res["fp8_repair"] = measure_repair(jattn, ctx, w, dinp, args.rho, steps, warmup, ms_fp8)
+        out[name] = res
+        del dinp
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_e2e(jattn, ctx: Ctx, w, inp, steps, warmup, flops):
     """Public one-call API with host (pinned) buffers: H2D of the step's
     inputs, the path, D2H of the output, all inside the timed region."""
     host = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
     out_host = torch.empty(w.B, w.S, w.H, w.d, dtype=torch.bfloat16).pin_memory()
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = out_host.numel() * out_host.element_size()
-
-    def one():
-        jattn.joint_attention(host["qkv_txt"], host["qkv_img"], host["qkv_ref"], host["pos"], w.split, w.theta,
-                              out=out_host)
-
-    for _ in range(warmup):
-        one()
-    barrier()
-    torch.cuda.synchronize()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(steps):
-        one()
-    t1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
-    ms = max_over_ranks(t0.elapsed_time(t1) / steps)
-    return {"value": round(whole_job_tflops(world, flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
+    ms, _ = time_calls(ctx, lambda ev: jattn.joint_attention(host["qkv_txt"], host["qkv_img"], host["qkv_ref"],
+                                                             host["pos"], w.split, w.theta, out=out_host),
+                       steps, warmup)
+    return {"value": round(whole_job_tflops(flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
             "api": "jattn.joint_attention -> jattn_joint_attention_host (C ABI, pinned host in/out, "
                    "copies pipelined with the kernels in (batch entry, 2-head) chunks on copy streams)"}
 
 
+# --------------------------------------------------------------------------- N > 1
+
+def run_partition(args, rank, world, local):
+    """The page's multi-GPU arrangement on `world` ranks: cfg_size x
+    ulysses_size (batch entries over rank groups, each entry's sequence over
+    its group), the whole batch fixed (strong scaling)."""
+    import datetime
+    import torch.distributed as dist
+    from diffusion_transformer_joint_jattn_b200 import jattn, ulysses
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+    ctx = Ctx(dev, world)
+    w = W.BY_NAME[args.workload]
+    lens = [w.S_txt, w.S_img, w.S_ref]
+    cfg, uly = ulysses.cfg_ulysses_layout(world, w.B, w.H, [n for n in lens if n])
+    groups = [dist.new_group(g) for g in ulysses.cfg_ulysses_groups(world, cfg, uly)]
+    bsl, g, r = ulysses.rank_work(rank, w.B, cfg, uly)
+    inp = W.make_inputs(w, seed=0)
+    streams = [None if t is None else t[bsl] for t in (inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"])]
+    shards = [None if t is None else t.to(dev) for t in ulysses.shard_streams(streams, uly, r)]
+    pos = inp["pos"].to(dev)
+
+    def step(ev):
+        ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g])
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms, _ = time_calls(ctx, step, args.steps, args.warmup)
+    clocks = sampler.stop()
+    code, bits = jattn.device_status(clear=True)
+    if code != jattn.OK:
+        raise RuntimeError(f"device status {code} bits {bits} on rank {rank}")
+    line = {
+        "metric": METRIC, "value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "d": w.d,
+                   "path": "bf16 in/out, fp16 MMA operands; ulysses_attention (NCCL all-to-all, rope, forward, "
+                           "all-to-all) per rank",
+                   "l2": "inputs larger than L2",
+                   "parallelism": f"cfg{cfg} x ulysses{uly}"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.barrier()
+    for grp in groups:
+        dist.destroy_process_group(grp)
+    dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- oracle on the host
+
 def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
     """Run the FP64 oracle on `heads` (b, h) pairs x `rows_per_head` query
-    rows of workload w.  Returns (seconds, flops)."""
+    rows of workload w.  Returns (seconds, flops, worker threads)."""
     import oracle
     from threadpoolctl import threadpool_limits
     sub = w.with_batch_heads(B=1, H=heads)
@@ -390,7 +477,7 @@ def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
     rows = W.sample_rows(sub, rows_per_head, seed)
     # One worker thread per host core, each with a single-threaded BLAS, so
     # the threads used are exactly `workers`.
-    workers = max(1, os.cpu_count() or 1)
+    workers = host_workers()
     with threadpool_limits(1):
         t = time.perf_counter()
         oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], sub.split, sub.theta,
@@ -410,52 +497,54 @@ def round_heads(w, n: float, workers: int) -> int:
     return int(max(1, min(w.B * w.H, -(-int(math.ceil(n)) // workers) * workers)))
 
 
-def cpu_baseline(w, target_s: float = 12.0):
-    # Calibrate on a small sample, then size the sample for ~target_s seconds.
-    # The small sample carries per-head fixed costs (rotating every key), so
-    # the first estimate runs short: rescale once more from the real run.
+def sample_shape(w, target_s: float):
+    """(heads, rows) of one oracle sample of about ``target_s`` seconds: one
+    head per worker thread, rows fitted from two timed probes (a fixed cost
+    per head -- rotating its keys -- plus a cost per row)."""
     workers = host_workers()
     heads = round_heads(w, 1, workers)
-    dt, fl, _ = oracle_sample(w, 128, heads)
-    rate = fl / dt
-    rows = int(max(128, min(w.S, target_s * rate / (4 * heads * w.S * w.d))))
-    dt, fl, workers = oracle_sample(w, rows, heads)
-    for _ in range(3):
-        if dt >= 0.6 * target_s or (rows >= w.S and heads >= w.B * w.H):
-            break
-        grow = target_s / max(dt, 1e-3)
-        if rows < w.S:
-            rows = int(min(w.S, rows * grow))
-        else:
-            heads = round_heads(w, max(heads + 1, heads * grow), workers)
-        dt, fl, workers = oracle_sample(w, rows, heads)
+    r0, r1 = min(64, w.S), min(256, w.S)
+    t0, _, _ = oracle_sample(w, r0, heads)
+    if r1 == r0:
+        return heads, r0
+    t1, _, _ = oracle_sample(w, r1, heads)
+    per_row = max((t1 - t0) / (r1 - r0), 1e-9)
+    fixed = max(t0 - per_row * r0, 0.0)
+    rows = int((target_s - fixed) / per_row)
+    return heads, int(max(32, min(w.S, rows)))
+
+
+def cpu_baseline(w, target_s: float = ORACLE_SAMPLE_S, samples: int = 2):
+    """The FP64 oracle on the host cores, on `samples` samples of the shape
+    the reference arm times per step."""
+    heads, rows = sample_shape(w, target_s)
+    dts, fl, workers = [], 0, host_workers()
+    for i in range(samples):
+        dt, fl, workers = oracle_sample(w, rows, heads, seed=i)
+        dts.append(dt)
+    dt = float(np.mean(dts))
     return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": workers, "blas_threads_per_worker": 1,
             "kind": "oracle",
-            "sample": f"{heads} heads x {rows} sampled query rows of {w.name} (S={w.S}, d={w.d}), "
-                      f"FP64 numpy oracle incl. RoPE, {dt:.1f} s"}
+            "sample": f"{heads} heads x {rows} sampled query rows of {w.name} (S={w.S}, d={w.d}), FP64 numpy "
+                      f"oracle incl. RoPE, mean of {samples} samples of {dt:.1f} s"}
 
 
 def run_reference(args, rank, world):
     if rank != 0:
         return
     w = W.BY_NAME[args.workload]
-    flops = 4 * w.B * w.H * w.S * w.S * w.d
-    heads = round_heads(w, 1, host_workers())
-    dt, fl, workers = oracle_sample(w, 128, heads)
-    rate = fl / dt
-    steps_budget_s = 150.0
-    per_step_s = max(1.0, steps_budget_s / max(1, args.steps + args.warmup))
-    rows = int(max(32, min(w.S, per_step_s * rate / (4 * heads * w.S * w.d))))
-    times = []
+    per_step_s = min(ORACLE_SAMPLE_S, max(0.5, 150.0 / max(1, args.steps + args.warmup)))
+    heads, rows = sample_shape(w, per_step_s)
+    times, fl, workers = [], 0, host_workers()
     for i in range(args.warmup + args.steps):
         dt, fl, workers = oracle_sample(w, rows, heads, seed=i)
         if i >= args.warmup:
             times.append(dt)
     sec = float(np.mean(times))
     value = fl / sec / 1e12
-    ms_full = flops / (fl / sec) * 1e3
+    ms_full = w.flops / (fl / sec) * 1e3
     line = {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_full, 1), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms_full, 1), "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "d": w.d,
                        "note": "each step = FP64 oracle on %d heads x %d sampled rows; ms_per_step extrapolated "

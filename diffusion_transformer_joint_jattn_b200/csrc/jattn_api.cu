@@ -24,14 +24,19 @@ constexpr int kMaxDevices = 64;
 
 uint32_t* status_ptr() {
   static uint32_t* ptrs[kMaxDevices] = {};
+  static unsigned long long ctx_ids[kMaxDevices] = {};
   static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  // Looked up again when the context changed (a cudaDeviceReset in between)
+  // or none was current yet (the lookup itself initialises it).
+  const unsigned long long ctx = jattn::current_context_id();
   std::lock_guard<std::mutex> lock(mu);
-  if (ptrs[dev] == nullptr) {
+  if (ptrs[dev] == nullptr || ctx == 0 || ctx_ids[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status_word) != cudaSuccess) return nullptr;
     ptrs[dev] = static_cast<uint32_t*>(p);
+    ctx_ids[dev] = jattn::current_context_id();
   }
   return ptrs[dev];
 }
@@ -52,6 +57,9 @@ EncodeTiledFn encode_fn() {
   });
   return fn;
 }
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -175,6 +183,32 @@ RepairLayout repair_layout(const jattn_shape* shape, int n) {
 }
 
 }  // namespace
+
+namespace jattn {
+
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
+}  // namespace jattn
 
 extern "C" {
 
@@ -388,6 +422,8 @@ jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits) {
   if (w & JATTN_DEV_RANGE) return JATTN_ERR_RANGE;
   return JATTN_OK;
 }
+
+jattn_status jattn_last_device_status(void* stream) { return jattn_device_status(stream, 0, nullptr); }
 
 jattn_status jattn_selftest_wait_timeout(int32_t limit_ms, void* stream) {
   if (limit_ms < 1 || limit_ms > 10000) return JATTN_ERR_INVALID_ARG;

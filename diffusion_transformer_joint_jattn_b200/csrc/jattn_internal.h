@@ -89,4 +89,10 @@ int fwd_kv_rows();
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st);
 
+// Unique id of the calling thread's current CUDA context (0 when there is
+// none or it cannot be read).  Device addresses of file-scope __device__
+// variables are cached per context: a cudaDeviceReset makes a new context,
+// whose id differs, and the address is looked up again.
+unsigned long long current_context_id();
+
 }  // namespace jattn

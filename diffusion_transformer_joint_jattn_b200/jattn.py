@@ -36,7 +36,7 @@ _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_fp8_repair",
            "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc",
            "jattn_joint_attention_host", "jattn_joint_attention_host_workspace", "jattn_fwd_bf16", "jattn_fwd_fp8",
-           "jattn_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
+           "jattn_device_status", "jattn_last_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
 
@@ -80,6 +80,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
+    lib.jattn_last_device_status.argtypes = [vp]
     lib.jattn_selftest_wait_timeout.argtypes = [i32, vp]
     lib.jattn_status_string.argtypes = [i32]
     lib.jattn_status_string.restype = ctypes.c_char_p
@@ -121,6 +122,60 @@ def _dev(t: torch.Tensor, name: str, dtype=None):
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _dev_shape(t: torch.Tensor, name: str, dtype, shape):
+    """``t`` must be a contiguous CUDA tensor of ``dtype`` and ``shape``: the
+    C ABI sees only a pointer, so a wrong size would become an out-of-bounds
+    device access."""
+    _dev(t, name, dtype)
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _check_repair_args(B, H, S, d, n, dev, o, lse, repaired, norm_w):
+    """Device, dtype and size checks of the FP8-with-repair outputs and norm
+    weights, before the call."""
+    for name, t in (("o", o), ("lse", lse), ("repaired", repaired), ("norm_w", norm_w)):
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} must be on {dev}, got {t.device}")
+    if o is not None:
+        _dev_shape(o, "o", torch.bfloat16, (B, S, H, d))
+    if lse is not None:
+        _dev_shape(lse, "lse", torch.float32, (B, H, S))
+    if repaired is not None:
+        _dev_shape(repaired, "repaired", torch.int32, (B, H, n))
+    if norm_w is not None:
+        _dev_shape(norm_w, "norm_w", torch.float32, (3, 2, d))
+
+
+def _streams(parts):
+    """Validate the per-stream QKV tensors [B, S_part, 3, H, d] (bf16, CUDA,
+    contiguous, one B / H / d for all) and return (B, H, d, [S_txt, S_img, S_ref])."""
+    ref = next((t for t in parts if t is not None), None)
+    if ref is None:
+        raise ValueError("at least one of qkv_txt, qkv_img, qkv_ref must be given")
+    if ref.dim() != 5:
+        raise ValueError(f"qkv streams must be [B, S, 3, H, d], got {tuple(ref.shape)}")
+    B, _, _, H, d = ref.shape
+    lens = []
+    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
+        if t is None:
+            lens.append(0)
+            continue
+        _dev(t, name, torch.bfloat16)
+        if t.dim() != 5 or t.shape[0] != B or t.shape[2] != 3 or t.shape[3] != H or t.shape[4] != d:
+            raise ValueError(f"{name} must be [B, S, 3, H, d], got {tuple(t.shape)}")
+        if t.device != ref.device:
+            raise ValueError(f"{name} must be on {ref.device}, got {t.device}")
+        lens.append(t.shape[1])
+    return B, H, d, lens
+
+
+def _positions(pos, S, dev):
+    _dev_shape(pos, "pos", torch.int32, (S, 3))
+    if pos.device != dev:
+        raise ValueError(f"pos must be on {dev}, got {pos.device}")
+
+
 def make_shape(B, H, S_txt, S_img, S_ref, d) -> Shape:
     return Shape(B, H, S_txt, S_img, S_ref, d)
 
@@ -141,18 +196,9 @@ def rope_qkv(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float 
     lib = load()
     parts = [qkv_txt, qkv_img, qkv_ref]
     ref = next(t for t in parts if t is not None)
-    B, _, _, H, d = ref.shape
-    lens = []
-    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
-        if t is None:
-            lens.append(0)
-            continue
-        _dev(t, name, torch.bfloat16)
-        if t.dim() != 5 or t.shape[0] != B or t.shape[2] != 3 or t.shape[3] != H or t.shape[4] != d:
-            raise ValueError(f"{name} must be [B, S, 3, H, d], got {tuple(t.shape)}")
-        lens.append(t.shape[1])
+    B, H, d, lens = _streams(parts)
     S = sum(lens)
-    _dev(pos, "pos", torch.int32)
+    _positions(pos, S, ref.device)
     code = _NAME_CODE[out_dtype] if isinstance(out_dtype, str) else _DTYPE_CODE[out_dtype]
     odt = _CODE_DTYPE[code]
     if out is None:
@@ -163,6 +209,10 @@ def rope_qkv(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float 
         scales = torch.empty(3, B, H, n_blocks(S), dtype=torch.float32, device=dev) if code == E4M3 else None
     else:
         q, k, v, scales = out
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _dev_shape(t, name, odt, (B, H, S, d))
+        if code == E4M3:
+            _dev_shape(scales, "scales", torch.float32, (3, B, H, n_blocks(S)))
     sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
     shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
     if norm_w is None:
@@ -183,12 +233,16 @@ def quant_fp8(x: torch.Tensor, out=None, stream=None):
     """Per-block e4m3 quantisation of a [B, H, S, d] fp16/bf16 tensor."""
     lib = load()
     _dev(x, "x")
+    if x.dim() != 4 or x.dtype not in (torch.bfloat16, torch.float16):
+        raise ValueError(f"x must be a bf16 / fp16 [B, H, S, d] tensor, got {x.dtype} {tuple(x.shape)}")
     B, H, S, d = x.shape
     if out is None:
         x8 = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=x.device)
         scales = torch.empty(B, H, n_blocks(S), dtype=torch.float32, device=x.device)
     else:
         x8, scales = out
+        _dev_shape(x8, "x8", torch.float8_e4m3fn, (B, H, S, d))
+        _dev_shape(scales, "scales", torch.float32, (B, H, n_blocks(S)))
     shape = make_shape(B, H, S, 0, 0, d)
     _check(lib.jattn_quant_fp8(ctypes.byref(shape), _DTYPE_CODE[x.dtype], _ptr(x), _ptr(x8), _ptr(scales),
                                _stream(stream)), "jattn_quant_fp8")
@@ -198,17 +252,23 @@ def quant_fp8(x: torch.Tensor, out=None, stream=None):
 def _fwd_outputs(B, H, S, d, dev, o, lse, want_lse):
     if o is None:
         o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=dev)
+    else:
+        _dev_shape(o, "o", torch.bfloat16, (B, S, H, d))
     if lse is None and want_lse:
         lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
+    elif lse is not None:
+        _dev_shape(lse, "lse", torch.float32, (B, H, S))
     return o, lse
 
 
 def fwd_bf16(q, k, v, o=None, lse=None, want_lse=False, softmax_scale: float = 0.0, stream=None):
     """O = softmax(Q K^T * scale) V for fp16/bf16 [B, H, S, d] operands."""
     lib = load()
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _dev(t, n, q.dtype)
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, H, S, d], got {tuple(q.shape)}")
     B, H, S, d = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_shape(t, n, q.dtype, (B, H, S, d))
     o, lse = _fwd_outputs(B, H, S, d, q.device, o, lse, want_lse)
     shape = make_shape(B, H, S, 0, 0, d)
     _check(lib.jattn_fwd_bf16(ctypes.byref(shape), _DTYPE_CODE[q.dtype], _ptr(q), _ptr(k), _ptr(v), _ptr(o),
@@ -220,10 +280,12 @@ def fwd_fp8(q8, k8, v8, scales, o=None, lse=None, want_lse=False, softmax_scale:
     """Attention forward on e4m3 [B, H, S, d] operands with fp32 block scales
     [3, B, H, ceil(S/128)]."""
     lib = load()
-    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
-        _dev(t, n, torch.float8_e4m3fn)
-    _dev(scales, "scales", torch.float32)
+    if q8.dim() != 4:
+        raise ValueError(f"q8 must be [B, H, S, d], got {tuple(q8.shape)}")
     B, H, S, d = q8.shape
+    for n, t in (("q8", q8), ("k8", k8), ("v8", v8)):
+        _dev_shape(t, n, torch.float8_e4m3fn, (B, H, S, d))
+    _dev_shape(scales, "scales", torch.float32, (3, B, H, n_blocks(S)))
     o, lse = _fwd_outputs(B, H, S, d, q8.device, o, lse, want_lse)
     shape = make_shape(B, H, S, 0, 0, d)
     _check(lib.jattn_fwd_fp8(ctypes.byref(shape), _ptr(q8), _ptr(k8), _ptr(v8), _ptr(scales), _ptr(o),
@@ -237,6 +299,12 @@ def device_status(clear: bool = True, stream=None):
     bits = ctypes.c_uint32(0)
     code = lib.jattn_device_status(_stream(stream), int(clear), ctypes.byref(bits))
     return code, bits.value
+
+
+def last_device_status(stream=None) -> int:
+    """jattn_last_device_status: wait for ``stream``'s work, return the
+    device status word's code without clearing it."""
+    return load().jattn_last_device_status(_stream(stream))
 
 
 def selftest_wait_timeout(limit_ms: int = 50, stream=None):
@@ -269,17 +337,10 @@ def fwd_fp8_repair(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: 
     lib = load()
     parts = [qkv_txt, qkv_img, qkv_ref]
     ref = next(t for t in parts if t is not None)
-    B, _, _, H, d = ref.shape
-    lens = []
-    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
-        if t is None:
-            lens.append(0)
-            continue
-        _dev(t, name, torch.bfloat16)
-        lens.append(t.shape[1])
+    B, H, d, lens = _streams(parts)
     S = sum(lens)
-    _dev(pos, "pos", torch.int32)
     dev = ref.device
+    _positions(pos, S, dev)
     n = repair_count(B, H, *lens, d, rho)
     need = repair_workspace_bytes(B, H, *lens, d, rho)
     if workspace is None:
@@ -289,8 +350,10 @@ def fwd_fp8_repair(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: 
     if want_lse and lse is None:
         lse = torch.empty(B, H, S, dtype=torch.float32, device=dev)
     rep = torch.empty(B, H, n, dtype=torch.int32, device=dev) if want_repaired else None
-    if norm_w is not None:
-        _dev(norm_w, "norm_w", torch.float32)
+    _check_repair_args(B, H, S, d, n, dev, o, lse, rep, norm_w)
+    _dev(workspace, "workspace", torch.uint8)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace must hold at least {need} bytes, got {workspace.numel()}")
     sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
     shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
     _check(lib.jattn_fwd_fp8_repair(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
@@ -319,13 +382,15 @@ def fwd_fp8_repair_noalloc(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int],
     lib = load()
     parts = [qkv_txt, qkv_img, qkv_ref]
     ref = next(t for t in parts if t is not None)
-    B, _, _, H, d = ref.shape
-    lens = [0 if t is None else t.shape[1] for t in parts]
-    for name, t in zip(("qkv_txt", "qkv_img", "qkv_ref"), parts):
-        if t is not None:
-            _dev(t, name, torch.bfloat16)
-    _dev(pos, "pos", torch.int32)
-    _dev(o, "o", torch.bfloat16)
+    B, H, d, lens = _streams(parts)
+    S = sum(lens)
+    _positions(pos, S, ref.device)
+    n = repair_count(B, H, *lens, d, rho)
+    if o is None:
+        raise ValueError("o must be given: this entry point allocates nothing")
+    _check_repair_args(B, H, S, d, n, ref.device, o, lse, repaired, norm_w)
+    if repaired is not None and n == 0:
+        repaired = None
     sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
     shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
     _check(lib.jattn_fwd_fp8_repair_noalloc(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref),

@@ -137,3 +137,31 @@ def shard_streams(streams: Sequence[Optional[torch.Tensor]], P: int, r: int):
         n = S_s // P
         out.append(t[:, r * n:(r + 1) * n].contiguous())
     return out
+
+
+def cfg_ulysses_layout(world: int, B: int, H: int, lens: Sequence[int]) -> Tuple[int, int]:
+    """(cfg_size, ulysses_size) for ``world`` ranks, as the page's multi-GPU
+    mode arranges them: the classifier-free-guidance branches (batch entries)
+    on separate rank groups when the batch splits evenly, the sequence of
+    each branch over the ranks of its group.  ulysses_size must divide H and
+    every stream's token count."""
+    cfg = 2 if world % 2 == 0 and B % 2 == 0 else 1
+    uly = world // cfg
+    if H % uly or any(n % uly for n in lens):
+        raise ValueError(f"{world} ranks: ulysses size {uly} must divide H = {H} and the stream lengths {list(lens)}")
+    return cfg, uly
+
+
+def cfg_ulysses_groups(world: int, cfg: int, uly: int):
+    """Rank lists of the Ulysses groups: group g holds ranks [g*uly, (g+1)*uly)
+    and serves batch entries [g*B/cfg, (g+1)*B/cfg)."""
+    if cfg * uly != world:
+        raise ValueError("cfg_size * ulysses_size must equal the world size")
+    return [list(range(g * uly, (g + 1) * uly)) for g in range(cfg)]
+
+
+def rank_work(rank: int, B: int, cfg: int, uly: int) -> Tuple[slice, int, int]:
+    """(batch slice, Ulysses group index, rank inside the group) of ``rank``."""
+    g, r = divmod(rank, uly)
+    nb = B // cfg
+    return slice(g * nb, (g + 1) * nb), g, r

@@ -33,7 +33,8 @@
  *     returns JATTN_ERR_CUDA.
  *   - Errors found on the device (a pipeline wait that ran out of time, a
  *     value out of the 16-bit output range) are recorded in a per-device
- *     status word; read it with jattn_device_status().  No kernel traps.
+ *     status word; read it with jattn_last_device_status() (or
+ *     jattn_device_status(), which can also clear it).  No kernel traps.
  *   - No C++ exception crosses this interface.
  */
 #ifndef JATTN_H_
@@ -204,18 +205,30 @@ jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt,
                                   int32_t* repaired, float softmax_scale, void* stream);
 
 /*
- * jattn_fwd_fp8_repair for callers that cannot allocate device memory: the
- * workspace is a file-scope device array of JATTN_NOALLOC_SCRATCH_BYTES
- * inside the library, reserved when a process first calls this function on a
- * device (its address is looked up once per device).  The library makes no
- * allocation on this path.
+ * jattn_fwd_fp8_repair for callers that cannot allocate device memory.  (No
+ * counterpart on the page: this is an interface for integrators.)  Some
+ * callers may not call cudaMalloc at all: a plug-in whose host framework owns
+ * every device allocation, code running inside a stream capture whose memory
+ * policy forbids allocation, or a latency-bound loop that must not block on
+ * the allocator.  They pass inputs and outputs as usual; the scratch the path
+ * needs is a file-scope device array of JATTN_NOALLOC_SCRATCH_BYTES inside
+ * the library.
+ *   Memory: with the CUDA runtime's default lazy module loading the array is
+ *   reserved on a device when a process first calls this function there;
+ *   with CUDA_MODULE_LOADING=EAGER every process that loads the library
+ *   reserves it on each device when its context is created.  The device holds
+ *   it until the process exits.  The path itself allocates nothing.
+ *   Set-up: the array's device address is looked up on the first call on a
+ *   device (make that call before any stream capture) and looked up again if
+ *   the device's context changed (after a cudaDeviceReset).
  *   Arguments: as jattn_fwd_fp8_repair without workspace / workspace_bytes.
  *   Errors: as jattn_fwd_fp8_repair; JATTN_ERR_UNSUPPORTED when
  *   jattn_fwd_fp8_repair_workspace(shape, rho) exceeds the array (checked
- *   before anything is launched), JATTN_ERR_CUDA if the array cannot be
- *   mapped.
- *   Calls on one device share the array: they must not overlap in time (use
- *   one stream per device, or serialise).
+ *   before anything is launched), JATTN_ERR_CUDA if the array's address
+ *   cannot be looked up.
+ *   Calls on one device share the array and overwrite what the last call
+ *   left there: calls that overlap on the GPU race (use one stream per
+ *   device, or serialise them).
  */
 #define JATTN_NOALLOC_SCRATCH_BYTES ((size_t)640 << 20)
 jattn_status jattn_fwd_fp8_repair_noalloc(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
@@ -247,6 +260,16 @@ jattn_status jattn_joint_attention_host(const jattn_shape* shape, const void* qk
                                         const void* qkv_ref, const int32_t* pos, float theta,
                                         const int32_t split[3], jattn_dtype path, void* o, float softmax_scale,
                                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The boundary's status query: wait for the work enqueued on `stream` so far,
+ * then return what the current device's status word records (JATTN_OK,
+ * JATTN_ERR_INTERNAL, JATTN_ERR_TIMEOUT or JATTN_ERR_RANGE, in that order of
+ * precedence) without clearing it.  JATTN_ERR_CUDA if the stream or the word
+ * cannot be read.  The word is per device: kernels of every stream and thread
+ * on the device record into it.
+ */
+jattn_status jattn_last_device_status(void* stream);
 
 /*
  * Synchronise `stream`, read the current device's status word and return

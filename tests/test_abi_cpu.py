@@ -196,3 +196,18 @@ def test_quant_rejects_bad_arguments():
 
 def test_selftest_rejects_bad_limit():
     assert jattn.load().jattn_selftest_wait_timeout(0, None) == jattn.ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    """The binding's copy of JATTN_NOALLOC_SCRATCH_BYTES equals the header's
+    macro (the oversize tests size their inputs from the binding's copy)."""
+    text = open(HEADER).read()
+    m = re.search(r"#define\s+JATTN_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)", text)
+    assert m is not None
+    assert int(m.group(1)) << int(m.group(2)) == jattn.NOALLOC_SCRATCH_BYTES
+
+
+def test_last_device_status_is_exported():
+    lib = jattn.load()
+    assert hasattr(lib, "jattn_last_device_status")
+    assert "jattn_last_device_status" in declared_symbols()

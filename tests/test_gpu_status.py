@@ -12,9 +12,13 @@ pytestmark = pytest.mark.gpu
 def test_bounded_wait_times_out_and_reports(cuda_device):
     jattn.device_status(clear=True)
     jattn.selftest_wait_timeout(50)
+    # the boundary's query reports it without clearing the word
+    assert jattn.last_device_status() == jattn.ERR_TIMEOUT
+    assert jattn.last_device_status() == jattn.ERR_TIMEOUT
     code, bits = jattn.device_status(clear=True)
     assert code == jattn.ERR_TIMEOUT and bits & jattn.DEV_TIMEOUT
     # the status is cleared and the context still runs work
     assert jattn.device_status(clear=False) == (jattn.OK, 0)
+    assert jattn.last_device_status() == jattn.OK
     x = torch.ones(4, device=cuda_device)
     assert float((x * 2).sum()) == 8.0

@@ -67,16 +67,17 @@ def test_noalloc_makes_no_allocation(cuda_device):
 
 def test_noalloc_refuses_oversize_inputs(cuda_device):
     """i2i at 2048x2048 (S = 33280, B = 2, H = 24) needs ~1 GB of workspace,
-    more than the array: refused on the host, outputs untouched."""
+    more than the array: refused on the host before anything is launched.
+    Every tensor pointer is NULL, so even if the size check stopped coming
+    first, the call would end in the argument checks (INVALID_ARG) and never
+    reach a kernel."""
     w = W.BY_NAME["i2i_2048_base"]
     need = jattn.repair_workspace_bytes(w.B, w.H, w.S_txt, w.S_img, w.S_ref, w.d, 0.005)
     assert need > jattn.NOALLOC_SCRATCH_BYTES
     lib = jattn.load()
     shape = jattn.make_shape(w.B, w.H, w.S_txt, w.S_img, w.S_ref, w.d)
     sp = (jattn.ctypes.c_int32 * 3)(*w.split)
-    o = torch.full((4,), 7.0, device=cuda_device)
-    fake = 1 << 20                              # never dereferenced: the size check comes first
-    code = lib.jattn_fwd_fp8_repair_noalloc(jattn.ctypes.byref(shape), fake, fake, None, fake, w.theta, sp, None,
-                                            1e-6, 0.005, fake, None, None, 0.0, None)
+    code = lib.jattn_fwd_fp8_repair_noalloc(jattn.ctypes.byref(shape), None, None, None, None, w.theta, sp, None,
+                                            1e-6, 0.005, None, None, None, 0.0, None)
     assert code == jattn.ERR_UNSUPPORTED
-    assert torch.all(o == 7.0)
+    assert jattn.device_status()[0] == jattn.OK
