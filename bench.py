@@ -213,9 +213,18 @@ def path_step(jattn, w, dinp, path: str, dev, stream):
     """Buffers and a step function for one whole-path step (prologue +
     forward) of workload w; the step records 3 events when given them."""
     B, H, S, d = w.B, w.H, w.S, w.d
+    ws = None
     if path == "bf16":
         q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
         bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
+    elif path == "bf16_hp":
+        q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
+        bufs = (q, torch.empty_like(q), torch.empty_like(q),
+                torch.empty(3, B, H, jattn.n_blocks(S), dtype=torch.float32, device=dev),
+                torch.empty(B, H, S, jattn.CORR_COLS, dtype=torch.float16, device=dev),
+                torch.empty(B, H, S, jattn.CORR_COLS, dtype=torch.float16, device=dev))
+        ws = torch.empty(jattn.rope_qkv_hp_workspace_bytes(B, H, w.S_txt, w.S_img, w.S_ref, d), dtype=torch.uint8,
+                         device=dev)
     else:
         q = torch.empty(B, H, S, d, dtype=torch.float8_e4m3fn, device=dev)
         bufs = (q, torch.empty_like(q), torch.empty_like(q),
@@ -225,12 +234,18 @@ def path_step(jattn, w, dinp, path: str, dev, stream):
     def step(ev):
         if ev is not None:
             ev[0].record(stream)
-        jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
-                       "fp16" if path == "bf16" else "e4m3", out=bufs, stream=stream)
+        if path == "bf16_hp":
+            jattn.rope_qkv_hp(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                              out=bufs, workspace=ws, stream=stream)
+        else:
+            jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                           "fp16" if path == "bf16" else "e4m3", out=bufs, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         if path == "bf16":
             jattn.fwd_bf16(bufs[0], bufs[1], bufs[2], o=o, stream=stream)
+        elif path == "bf16_hp":
+            jattn.fwd_bf16_hp(*bufs, o=o, stream=stream)
         else:
             jattn.fwd_fp8(bufs[0], bufs[1], bufs[2], bufs[3], o=o, stream=stream)
         if ev is not None:
@@ -273,6 +288,12 @@ def run_ours(args, rank, world, local):
     sampler.start()
     ms, pro_ms, fwd_ms, fwd_med, fwd_min = measure_path(jattn, ctx, w, dinp, "bf16", args.steps, args.warmup)
     clocks = sampler.stop()
+    msh, proh, fwdh, fwdh_med, fwdh_min = measure_path(jattn, ctx, w, dinp, "bf16_hp", args.steps, args.warmup)
+    hp = {"value": round(whole_job_tflops(flops, msh), 2), "unit": UNIT, "ms_per_step": round(msh, 4),
+          "prologue_ms": round(proh, 4), "fwd_ms": round(fwdh, 4), "fwd_ms_median": round(fwdh_med, 4),
+          "fwd_ms_min": round(fwdh_min, 4), "gpu_launches_per_step": 4,
+          "roofline": tensor_roofline(flops, fwdh, peaks, peak_src, False, None,
+                                      "attn_fwd_kernel<128, fp16 operands, high precision>")}
     fp8 = None
     if not args.no_fp8:
         ms8, pro8, fwd8, fwd8_med, fwd8_min = measure_path(jattn, ctx, w, dinp, "fp8", args.steps, args.warmup)
@@ -312,6 +333,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches": 2 * args.steps,
         "clocks": clocks,
     }
+    line["bf16_hp"] = hp
     if fp8 is not None:
         line["fp8"] = fp8
     line.update(extras)

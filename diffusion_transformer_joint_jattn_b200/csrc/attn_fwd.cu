@@ -54,7 +54,10 @@ constexpr float kRescaleThreshold = 8.0f;   // log2 units: P <= 2^8 before a res
 __host__ __device__ constexpr uint32_t col_s(int t) { return static_cast<uint32_t>(t) * 128u; }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
 
-template <int D, bool FP8>
+// HP: the high-precision 16-bit instance, which also stages one correction
+// tile (128 rows x 16 fp16 = 32 bytes, 32-byte swizzle) per query tile and
+// per K stage.
+template <int D, bool FP8, bool HP = false>
 struct Cfg {
   static constexpr int ES = FP8 ? 1 : 2;              // element bytes
   static constexpr int RB = D * ES;                   // row bytes
@@ -67,9 +70,10 @@ struct Cfg {
   static constexpr int MK = FP8 ? 32 : 16;            // K per MMA instruction
   static constexpr int QK_STEPS = RB / 32;            // 32 bytes of K per step
   static constexpr int PV_STEPS = BN / MK;
-  static constexpr int KS = TB >= 32768 ? 3 : 4;      // K ring stages
+  static constexpr int KS = TB >= 32768 ? (HP ? 2 : 3) : 4;   // K ring stages
   static constexpr int VS = TB >= 32768 ? 2 : 4;      // V ring stages
-  static constexpr int SMEM = (NQ + KS + VS) * TB + 2048;
+  static constexpr int CT = HP ? BM * 32 : 0;         // correction tile bytes
+  static constexpr int SMEM = (NQ + KS + VS) * TB + (NQ + KS) * CT + 2048;
 };
 
 struct __align__(8) Bars {
@@ -140,13 +144,19 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }
 
 // KIND: 0 = fp16 operands, 1 = bf16 operands, 2 = e4m3 operands.
-template <int D, int KIND>
+// HP (KIND 0 only): the high-precision 16-bit path -- per-block power-of-two
+// range scales of Q, K and V folded in like the e4m3 block scales, and each
+// logit tile completed by Qc . Kc^T over the correction tiles (tmQc, tmKc).
+template <int D, int KIND, bool HP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQc,
+                const __grid_constant__ CUtensorMap tmKc, const FwdParams p) {
   constexpr bool FP8 = KIND == 2;
+  constexpr bool SCALED = FP8 || HP;                   // per-block scales of Q, K and V
+  static_assert(!HP || KIND == 0, "the high-precision path has fp16 operands");
   constexpr uint32_t in_fmt = KIND == 1 ? 1u : 0u;   // f16 / bf16 (kind::f16); e4m3 (kind::f8f6f4)
-  using C = Cfg<D, FP8>;
+  using C = Cfg<D, FP8, HP>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzle atoms.
   const uint32_t raw_u32 = smem_u32(smem_raw);
@@ -154,7 +164,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   uint8_t* sQ = smem;                                  // NQ tiles
   uint8_t* sK = sQ + NQ * C::TB;
   uint8_t* sV = sK + C::KS * C::TB;
-  Bars* bar = reinterpret_cast<Bars*>(sV + C::VS * C::TB);
+  uint8_t* sQc = sV + C::VS * C::TB;                   // HP: NQ correction tiles, then KS
+  uint8_t* sKc = sQc + NQ * C::CT;
+  Bars* bar = reinterpret_cast<Bars*>(sKc + C::KS * C::CT);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -202,17 +214,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      mbar_arrive_expect_tx(&bar->q_full, NQ * C::TB);
-      for (int t = 0; t < NQ; ++t)
+      if constexpr (HP) {
+        tma_prefetch_desc(&tmQc);
+        tma_prefetch_desc(&tmKc);
+      }
+      mbar_arrive_expect_tx(&bar->q_full, NQ * (C::TB + C::CT));
+      for (int t = 0; t < NQ; ++t) {
         for (int x = 0; x < C::NBOX; ++x)
           tma_load_3d(&tmQ, &bar->q_full, sQ + t * C::TB + x * C::BOXB, x * C::BOX_ELEMS, (qp * NQ + t) * BM, bh);
+        if constexpr (HP) tma_load_3d(&tmQc, &bar->q_full, sQc + t * C::CT, 0, (qp * NQ + t) * BM, bh);
+      }
       int nk = 0, nv = 0;
       for (int j = 0; j < n_kv; ++j) {
         const int ks = j % C::KS;
         if (!mbar_wait(&bar->k_empty[ks], ((j / C::KS) & 1) ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(&bar->k_full[ks], C::TB);
+        mbar_arrive_expect_tx(&bar->k_full[ks], C::TB + C::CT);
         for (int x = 0; x < C::NBOX; ++x)
           tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
+        if constexpr (HP) tma_load_3d(&tmKc, &bar->k_full[ks], sKc + ks * C::CT, 0, j * BN, bh);
         nk = j + 1;
         const int vs = j % C::VS;
         if (!mbar_wait(&bar->v_empty[vs], ((j / C::VS) & 1) ^ 1, ctl)) break;
@@ -243,6 +262,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const uint64_t bdesc = smem_desc(kbase + off, 16, 8 * C::SWB, C::SWMODE);
           if constexpr (FP8) mma_f8_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, kk > 0);
           else mma_f16_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, kk > 0);
+        }
+        if constexpr (HP) {
+          // the low-order terms of the selected channels: one 16-deep step
+          const uint64_t adesc = smem_desc(smem_u32(sQc) + t * C::CT, 16, 256, kSwizzle32B);
+          const uint64_t bdesc = smem_desc(smem_u32(sKc) + ks * C::CT, 16, 256, kSwizzle32B);
+          mma_f16_ss(tmem + col_s(t), adesc, bdesc, idesc_qk, 1);
         }
         any_mma = true;
       };
@@ -324,7 +349,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     float sq = 1.f, max_sv = 1.f;
     const float* sc_k = nullptr;
     const float* sc_v = nullptr;
-    if constexpr (FP8) {
+    if constexpr (SCALED) {
       const size_t nb = static_cast<size_t>(p.n_tiles);
       const size_t bhn = static_cast<size_t>(bh) * nb;
       const size_t plane = static_cast<size_t>(p.B) * p.H * nb;
@@ -338,19 +363,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       max_sv = mv > 0.f ? mv : 1.f;
     }
     // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
-    // exceeds the e4m3 range while p <= 2^8.
-    const float p8_log2 = 8.8073549220576042f - kRescaleThreshold;   // log2(448) - 8
-    // FP8: the K / V block scales of the next tile are fetched one tile ahead
-    // so that their load latency stays off the S -> P chain.
+    // exceeds the e4m3 range while p <= 2^8.  HP: as p * (s_v,j / max s_v)
+    // (powers of two; at most 2^8 in fp16).
+    const float p8_log2 = FP8 ? 8.8073549220576042f - kRescaleThreshold : 0.f;   // log2(448) - 8
+    // The K / V block scales of the next tile are fetched one tile ahead so
+    // that their load latency stays off the S -> P chain.
     float sk_nxt = 0.f, sv_nxt = 0.f;
-    if constexpr (FP8) {
+    if constexpr (SCALED) {
       sk_nxt = sc_k[0];
       sv_nxt = sc_v[0];
     }
 
     for (int j = 0; j < n_kv; ++j) {
       float c_j = sl2, bias = 0.f;
-      if constexpr (FP8) {
+      if constexpr (SCALED) {
         c_j = sl2 * sq * sk_nxt;
         bias = __log2f(sv_nxt / max_sv) + p8_log2;
         if (j + 1 < n_kv) {
@@ -480,7 +506,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       }
       float ls = (acc0.x + acc0.y) + (acc1.x + acc1.y);
       if (n_left_out != 0.f) ls = fmaf(-n_left_out, ex2_approx(neg_m), ls);   // zero-logit keys left out
-      if constexpr (FP8) ls *= ex2_approx(-bias);
+      if constexpr (SCALED) ls *= ex2_approx(-bias);
       l_run += ls;
       tc_fence_before();
       mbar_arrive(&bar->p_full[t]);
@@ -491,7 +517,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       __syncwarp();
       tc_fence_after();
       float out_scale = 1.f / l_run;
-      if constexpr (FP8) out_scale *= max_sv * ex2_approx(-p8_log2);
+      if constexpr (SCALED) out_scale *= max_sv * ex2_approx(-p8_log2);
       float lse2 = m_run + __log2f(l_run);             // log2 units
       // Merge with a partial result over other keys already in o:
       // O = w_a O_a + w_b O_b with w = 2^(LSE_part - LSE), LSE = log2(2^a + 2^b).
@@ -553,16 +579,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
-template <int D, int KIND>
+template <int D, int KIND, bool HP = false>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                     cudaStream_t st) {
-  using C = Cfg<D, KIND == 2>;
+                     const CUtensorMap& tqc, const CUtensorMap& tkc, cudaStream_t st) {
+  using C = Cfg<D, KIND == 2, HP>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  auto kern = attn_fwd_kernel<D, KIND>;
+  auto kern = attn_fwd_kernel<D, KIND, HP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((p.n_tiles + NQ - 1) / NQ, p.B * p.H);
-  kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, p);
+  kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, tqc, tkc, p);
   return cudaGetLastError();
 }
 
@@ -587,13 +613,20 @@ int fwd_kv_rows() { return BN; }
 
 cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
-  if (in_bf16) return d == 128 ? launch_t<128, 1>(p, tq, tk, tv, st) : launch_t<64, 1>(p, tq, tk, tv, st);
-  return d == 128 ? launch_t<128, 0>(p, tq, tk, tv, st) : launch_t<64, 0>(p, tq, tk, tv, st);
+  if (in_bf16) return d == 128 ? launch_t<128, 1>(p, tq, tk, tv, tq, tk, st) : launch_t<64, 1>(p, tq, tk, tv, tq, tk, st);
+  return d == 128 ? launch_t<128, 0>(p, tq, tk, tv, tq, tk, st) : launch_t<64, 0>(p, tq, tk, tv, tq, tk, st);
+}
+
+cudaError_t launch_fwd_f16_hp(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const CUtensorMap& tqc, const CUtensorMap& tkc,
+                              cudaStream_t st) {
+  return d == 128 ? launch_t<128, 0, true>(p, tq, tk, tv, tqc, tkc, st)
+                  : launch_t<64, 0, true>(p, tq, tk, tv, tqc, tkc, st);
 }
 
 cudaError_t launch_fwd_fp8(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, cudaStream_t st) {
-  return d == 128 ? launch_t<128, 2>(p, tq, tk, tv, st) : launch_t<64, 2>(p, tq, tk, tv, st);
+  return d == 128 ? launch_t<128, 2>(p, tq, tk, tv, tq, tk, st) : launch_t<64, 2>(p, tq, tk, tv, tq, tk, st);
 }
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t st) {

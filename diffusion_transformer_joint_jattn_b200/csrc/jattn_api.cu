@@ -93,6 +93,22 @@ jattn_status make_map(CUtensorMap* m, const void* base, int BH, int S, int d, in
   return r == CUDA_SUCCESS ? JATTN_OK : JATTN_ERR_CUDA;
 }
 
+// [BH][S][16] fp16 correction rows; boxes of 16 x box_rows, 32-byte swizzle.
+jattn_status make_map_corr(CUtensorMap* m, const void* base, int BH, int S, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return JATTN_ERR_CUDA;
+  const int row_bytes = jattn::kCorrCols * 2;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(jattn::kCorrCols), static_cast<cuuint64_t>(S),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(row_bytes) * S};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(jattn::kCorrCols), static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? JATTN_OK : JATTN_ERR_CUDA;
+}
+
 float resolve_scale(float softmax_scale, int d) {
   return softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(static_cast<float>(d));
 }
@@ -100,7 +116,8 @@ float resolve_scale(float softmax_scale, int d) {
 jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img, const void* qkv_ref,
                          const int32_t* pos, float theta, const int32_t split[3], const float* norm_w, float eps,
                          jattn_dtype out_dtype, void* q, void* k, void* v, float* scales, void* stream,
-                         void* q16 = nullptr, float* score = nullptr) {
+                         void* q16 = nullptr, float* score = nullptr, float* pair_stat = nullptr,
+                         float* norm_r = nullptr) {
   jattn_status st = check_shape(shape);
   if (st != JATTN_OK) return st;
   if (split == nullptr || pos == nullptr || q == nullptr || k == nullptr || v == nullptr) return JATTN_ERR_INVALID_ARG;
@@ -140,6 +157,9 @@ jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const vo
   p.eps = eps;
   p.q16 = q16;
   p.score = score;
+  p.hp = pair_stat != nullptr ? 1 : 0;
+  p.pair_stat = pair_stat;
+  p.norm_r = norm_r;
   p.status = status_ptr();
   if (p.status == nullptr) return JATTN_ERR_CUDA;
   const int kind = out_dtype == JATTN_FP16 ? 0 : (out_dtype == JATTN_BF16 ? 1 : 2);
@@ -155,6 +175,25 @@ int repair_n(const jattn_shape* shape, float rho) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Scratch of the high-precision prologue: pair statistics, selected pairs,
+// RMSNorm row factors (each segment 256-byte aligned).
+struct HpLayout {
+  size_t pair_stat, sel, norm_r, total;
+};
+
+HpLayout hp_layout(const jattn_shape* shape) {
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const size_t S = total_S(shape), d = shape->d, nb = n_blocks(static_cast<int>(S));
+  HpLayout L{};
+  size_t off = 0;
+  auto seg = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+  L.pair_stat = seg(2 * BH * nb * (d / 2) * 4);
+  L.sel = seg(BH * jattn::kCorrPairs * 4);
+  L.norm_r = seg(2 * BH * S * 4);
+  L.total = off;
+  return L;
+}
 
 // Workspace segments, each 256-byte aligned, in this order.
 struct RepairLayout {
@@ -309,6 +348,83 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
   if ((st = make_map(&tk, k8, BH, p.S, shape->d, 1, kv_rows)) != JATTN_OK) return st;
   if ((st = make_map(&tv, v8, BH, p.S, shape->d, 1, kv_rows)) != JATTN_OK) return st;
   return jattn::launch_fwd_fp8(p, shape->d, tq, tk, tv, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? JATTN_OK
+             : JATTN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------- high-precision 16-bit path
+
+size_t jattn_rope_qkv_hp_workspace(const jattn_shape* shape) {
+  if (check_shape(shape) != JATTN_OK) return 0;
+  return hp_layout(shape).total;
+}
+
+jattn_status jattn_rope_qkv_hp(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                               const void* qkv_ref, const int32_t* pos, float theta, const int32_t split[3],
+                               const float* norm_w, float eps, void* q, void* k, void* v, float* scales, void* qc,
+                               void* kc, void* workspace, size_t workspace_bytes, void* stream) {
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  if (norm_w != nullptr && (!(eps > 0.f) || !std::isfinite(eps))) return JATTN_ERR_INVALID_ARG;
+  if (scales == nullptr || qc == nullptr || kc == nullptr || workspace == nullptr) return JATTN_ERR_INVALID_ARG;
+  const HpLayout L = hp_layout(shape);
+  if (workspace_bytes < L.total) return JATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return JATTN_ERR_ALIGNMENT;
+  if (!aligned16(qc) || !aligned16(kc) || !aligned16(scales)) return JATTN_ERR_ALIGNMENT;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* pair_stat = reinterpret_cast<float*>(ws + L.pair_stat);
+  float* norm_r = reinterpret_cast<float*>(ws + L.norm_r);
+  // 1. prologue: fp16 Q, K, V with power-of-two range scales, pair statistics
+  st = rope_common(shape, qkv_txt, qkv_img, qkv_ref, pos, theta, split, norm_w, eps, JATTN_FP16, q, k, v, scales,
+                   stream, nullptr, nullptr, pair_stat, norm_r);
+  if (st != JATTN_OK) return st;
+  // 2. pair selection and 3. correction rows
+  jattn::CorrParams c{};
+  const void* parts[3] = {qkv_txt, qkv_img, qkv_ref};
+  const int lens[3] = {shape->S_txt, shape->S_img, shape->S_ref};
+  for (int i = 0; i < 3; ++i) {
+    c.src[i] = static_cast<const __nv_bfloat16*>(parts[i]);
+    c.S_part[i] = lens[i];
+    c.split[i] = split[i];
+  }
+  c.B = shape->B;
+  c.H = shape->H;
+  c.BH = shape->B * shape->H;
+  c.S = total_S(shape);
+  c.d = shape->d;
+  c.nblk = n_blocks(c.S);
+  c.pos = pos;
+  c.theta = static_cast<double>(theta);
+  c.norm_w = norm_w;
+  c.norm_r = norm_w != nullptr ? norm_r : nullptr;
+  c.scales = scales;
+  c.pair_stat = pair_stat;
+  c.sel = reinterpret_cast<int32_t*>(ws + L.sel);
+  c.qc = qc;
+  c.kc = kc;
+  return jattn::launch_qk_correction(c, static_cast<cudaStream_t>(stream)) == cudaSuccess ? JATTN_OK
+                                                                                         : JATTN_ERR_CUDA;
+}
+
+jattn_status jattn_fwd_bf16_hp(const jattn_shape* shape, const void* q, const void* k, const void* v,
+                               const float* scales, const void* qc, const void* kc, void* o, float* lse,
+                               float softmax_scale, void* stream) {
+  if (scales == nullptr || qc == nullptr || kc == nullptr) return JATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(scales) & 3u) || !aligned16(qc) || !aligned16(kc)) return JATTN_ERR_ALIGNMENT;
+  jattn::FwdParams p{};
+  jattn_status st = fwd_common(shape, q, k, v, o, lse, softmax_scale, p);
+  if (st != JATTN_OK) return st;
+  p.scales = scales;
+  CUtensorMap tq, tk, tv, tqc, tkc;
+  const int BH = p.B * p.H;
+  const int kv_rows = jattn::fwd_kv_rows();
+  if ((st = make_map(&tq, q, BH, p.S, shape->d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map_corr(&tqc, qc, BH, p.S, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map_corr(&tkc, kc, BH, p.S, kv_rows)) != JATTN_OK) return st;
+  return jattn::launch_fwd_f16_hp(p, shape->d, tq, tk, tv, tqc, tkc, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
              ? JATTN_OK
              : JATTN_ERR_CUDA;
 }

@@ -22,6 +22,10 @@ struct RopeParams {
   float eps;                    // RMSNorm epsilon
   void* q16;                    // e4m3 output with token repair: also fp16 Q [B, H, S, d], else null
   float* score;                 // with token repair: [2][B, H, S], |k|^2 then |v|^2 per token, else null
+  int hp;                       // fp16 output of the high-precision path: power-of-two range scales in
+                                //   `scales` ([3][B][H][nblk]), pair statistics and norm factors below
+  float* pair_stat;             // hp: [2][B*H][nblk][d/2] max squared channel-pair norm over each block
+  float* norm_r;                // hp with norm_w: [2][B*H][S] RMSNorm factor of every Q / K row
   uint32_t* status;
 };
 
@@ -51,6 +55,30 @@ cudaError_t launch_repair_gather(const GatherParams& p, cudaStream_t st);
 cudaError_t launch_repair_select(float* score, int BH, int S, int n, int n_kv, int32_t* idx,
                                  uint32_t* kmask, cudaStream_t st);
 
+// High-precision 16-bit path: channel pairs per (b, h) whose rotated Q / K
+// values get an fp16 low part, and the columns of one correction row
+// (hi and lo of 2 * kCorrPairs channels).
+constexpr int kCorrPairs = 4;
+constexpr int kCorrCols = 4 * kCorrPairs;
+
+struct CorrParams {
+  const __nv_bfloat16* src[3];  // txt, img, ref streams [B, S_part, 3, H, d]
+  int S_part[3];
+  int B, H, BH, S, d, nblk;
+  const int32_t* pos;           // [S, 3]
+  double theta;
+  int split[3];
+  const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
+  const float* norm_r;          // with norm_w: [2][B*H][S] row factors written by the prologue
+  const float* scales;          // [3][B][H][nblk] power-of-two range scales written by the prologue
+  const float* pair_stat;       // [2][B*H][nblk][d/2] written by the prologue
+  int32_t* sel;                 // [B*H][kCorrPairs] selected pairs, ascending
+  void* qc;                     // fp16 [B*H][S][kCorrCols]: [hi | lo] of the selected Q channels
+  void* kc;                     // fp16 [B*H][S][kCorrCols]: [lo | hi] of the selected K channels
+};
+
+cudaError_t launch_qk_correction(const CorrParams& p, cudaStream_t st);
+
 struct QuantParams {
   const void* x;                // [BH, S, d] 16-bit
   void* x8;                     // [BH, S, d] e4m3
@@ -64,7 +92,7 @@ struct FwdParams {
   float scale_log2;             // softmax_scale * log2(e)
   __nv_bfloat16* o;             // [B, S, H, d]
   float* lse;                   // [B, H, S] or null
-  const float* scales;          // fp8: [3][B][H][n_tiles]
+  const float* scales;          // fp8 and the high-precision fp16 path: [3][B][H][n_tiles]
   const uint32_t* kmask;        // null, or [B*H][n_kv][4] words: bit set = key left out of this pass
   const float* lse_prev;        // null, or [B, H, S]: o already holds a partial result with this
                                 // LSE over other keys; the pass merges its own into o (and lse)
@@ -83,6 +111,12 @@ cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtens
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st);
 cudaError_t launch_fwd_fp8(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
                            const CUtensorMap& tv, cudaStream_t st);
+// High-precision 16-bit forward: fp16 operands with power-of-two block scales
+// in p.scales and the correction tiles described by tqc / tkc ([BH][S][16]
+// fp16, 32-byte swizzle, 128-row boxes).
+cudaError_t launch_fwd_f16_hp(const FwdParams& p, int d, const CUtensorMap& tq, const CUtensorMap& tk,
+                              const CUtensorMap& tv, const CUtensorMap& tqc, const CUtensorMap& tkc,
+                              cudaStream_t st);
 
 // Rows of the K / V tiles the forward kernels walk (the TMA box height).
 int fwd_kv_rows();

@@ -257,7 +257,9 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 // Shared-memory matrix descriptor (tcgen05 format): start address, leading
 // and stride byte offsets (all >> 4), descriptor version 1, swizzle mode in
-// bits [61, 64): 2 = 128-byte swizzle, 4 = 64-byte swizzle.
+// bits [61, 64): 2 = 128-byte swizzle, 4 = 64-byte swizzle, 6 = 32-byte
+// swizzle.
+constexpr uint32_t kSwizzle32B = 6u;
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes,
                                               uint32_t swizzle_mode) {
   uint64_t d = 0;

@@ -30,6 +30,7 @@
 
 #include "jattn.h"
 #include "jattn_internal.h"
+#include "rope_math.cuh"
 
 namespace jattn {
 
@@ -39,15 +40,6 @@ constexpr int kTok = JATTN_BLOCK;   // tokens per CTA (= FP8 scale block)
 constexpr int kTokPerThread = 4;
 
 enum OutKind { kOutF16 = 0, kOutBF16 = 1, kOutE4M3 = 2 };
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&x)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = __uint_as_float(w[i] << 16);
-    x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-  }
-}
 
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
@@ -70,42 +62,34 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-// Axis, index inside the axis span and span width of channel pair `pair`
-// (0 .. d/2-1); spans are laid out t, row, col.
-__device__ __forceinline__ void pair_axis(int pair, int n0, int n1, int n2, int& axis, int& i, int& n) {
-  if (pair < n0 / 2) { axis = 0; i = pair; n = n0; }
-  else if (pair < (n0 + n1) / 2) { axis = 1; i = pair - n0 / 2; n = n1; }
-  else { axis = 2; i = pair - (n0 + n1) / 2; n = n2; }
-}
-
-// cos/sin of pos_axis * theta^(-2i/n): the angle is formed and reduced to
-// [-pi, pi] in fp64, then rotated with the fp32 sincos.
-__device__ __forceinline__ void pair_cos_sin(int32_t pos_axis, int i, int n, double theta,
-                                             float& c, float& s) {
-  const double omega = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(n));
-  const double ang = static_cast<double>(pos_axis) * omega;
-  const double two_pi = 6.283185307179586476925286766559;
-  const double r = ang - rint(ang / two_pi) * two_pi;
-  sincosf(static_cast<float>(r), &s, &c);
-}
-
 // OUT: output kind.  D: head dimension.  NORM: RMSNorm Q and K first.
 // REPAIR (e4m3 output only): also write fp16 Q and the per-token repair score
 // |k|^2 + |v|^2 of the values that are quantised.
-template <int D, int OUT, bool NORM, bool REPAIR>
+// HP (fp16 output only), the high-precision 16-bit path: every (Q|K|V, head)
+// tile is stored scaled by a power of two 2^-e chosen from the tile's amax
+// so that nothing saturates (e = 0 unless the tile reaches past 65504; the
+// scale 2^e goes to p.scales, [3][B][H][nblk]); for Q and K the maximum
+// squared norm of every channel pair over the block's tokens goes to
+// p.pair_stat ([2][B*H][nblk][D/2]), and with NORM each row's RMSNorm factor
+// to p.norm_r ([2][B*H][S]), for the correction operands built afterwards.
+template <int D, int OUT, bool NORM, bool REPAIR, bool HP>
 __global__ void __launch_bounds__(D / 8 * kTok / kTokPerThread)
 rope_qkv_kernel(const RopeParams p) {
   constexpr int CG = D / 8;                           // 16-byte chunks per row
   constexpr int NT = CG * kTok / kTokPerThread;       // threads
   constexpr int ROWS_PER_PASS = kTok / kTokPerThread; // tokens covered by one pass
   constexpr int NWARP = NT / 32;
+  constexpr int NPAIR = D / 2;
   static_assert(CG <= 32 && 32 % CG == 0, "a row's lanes must sit inside one warp");
+  static_assert(!HP || OUT == kOutF16, "the high-precision path stores fp16");
   __shared__ float red[2][NWARP];
   __shared__ __align__(16) float wsm[NORM ? 6 * D : 4];   // [stream][q/k][D]
+  __shared__ __align__(16) float pst[HP ? 2 : 1][HP ? NWARP : 1][HP ? NPAIR : 4];   // pair statistics per warp
 
   const int tid = threadIdx.x;
   const int cg = tid % CG;
   const int trow = tid / CG;
+  const int warp = tid >> 5, lane = tid & 31;
   const int blk = blockIdx.x;
   const int b = blockIdx.y;
   const int H = p.H, S = p.S;
@@ -179,6 +163,7 @@ rope_qkv_kernel(const RopeParams p) {
     if (item + 1 < items) load_item(item + 1, nxt);
     if (item + 2 < items) prefetch_item_l2(item + 2);
     const int which = item / H, h = item % H;
+    const size_t row0 = (static_cast<size_t>(b) * H + h) * S;
 
     float x[kTokPerThread][8];
 #pragma unroll
@@ -189,26 +174,25 @@ rope_qkv_kernel(const RopeParams p) {
         // the row's other chunks sit in the CG consecutive lanes around it.
         float ss = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(x[i][e], x[i][e], ss);
+        for (int e = 0; e < 8; ++e) ss = __fmaf_rn(x[i][e], x[i][e], ss);
 #pragma unroll
         for (int o = CG / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float r = __frsqrt_rn(fmaf(ss, 1.0f / D, p.eps));
+        const float r = norm_factor(ss, D, p.eps);
         const float4* wv = reinterpret_cast<const float4*>(wsm + (stream[i] * 2 + which) * D + cg * 8);
         const float4 w0 = wv[0], w1 = wv[1];
         const float wr[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[i][e] = x[i][e] * r * wr[e];
+        for (int e = 0; e < 8; ++e) x[i][e] = norm_scale(x[i][e], r, wr[e]);
+        if constexpr (HP) {
+          if (cg == 0 && valid[i]) p.norm_r[static_cast<size_t>(which) * p.B * H * S + row0 + tok[i]] = r;
+        }
       }
       if (which < 2) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float a = x[i][2 * j], bb = x[i][2 * j + 1];
-          x[i][2 * j] = a * cs[i][j] - bb * sn[i][j];
-          x[i][2 * j + 1] = a * sn[i][j] + bb * cs[i][j];
-        }
+        for (int j = 0; j < 4; ++j) rotate_pair(x[i][2 * j], x[i][2 * j + 1], cs[i][j], sn[i][j], x[i][2 * j],
+                                                x[i][2 * j + 1]);
       }
     }
-    const size_t row0 = (static_cast<size_t>(b) * H + h) * S;
 
     if constexpr (REPAIR) {
       if (which == 0) {
@@ -275,6 +259,45 @@ rope_qkv_kernel(const RopeParams p) {
       if (tid == 0)
         p.scales[((static_cast<size_t>(which) * p.B + b) * H + h) * p.nblk + blk] = scale;
     } else {
+      float inv2e = 1.0f;
+      if constexpr (HP) {
+        // The tile's amax -> power-of-two range scale; for Q and K the
+        // per-pair maximum squared norm over the block's tokens.
+        float am = 0.f;
+#pragma unroll
+        for (int i = 0; i < kTokPerThread; ++i)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x[i][e]));
+        am = warp_max(am);
+        if (lane == 0) red[item & 1][warp] = am;
+        if (which < 2) {
+          float pn[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            pn[j] = 0.f;
+#pragma unroll
+            for (int i = 0; i < kTokPerThread; ++i)
+              pn[j] = fmaxf(pn[j], __fmaf_rn(x[i][2 * j], x[i][2 * j], __fmul_rn(x[i][2 * j + 1], x[i][2 * j + 1])));
+#pragma unroll
+            for (int o = CG; o < 32; o <<= 1) pn[j] = fmaxf(pn[j], __shfl_xor_sync(0xffffffffu, pn[j], o));
+          }
+          if (lane < CG)
+            *reinterpret_cast<float4*>(&pst[item & 1][warp][cg * 4]) = make_float4(pn[0], pn[1], pn[2], pn[3]);
+        }
+        __syncthreads();
+        am = 0.f;
+#pragma unroll
+        for (int w = 0; w < NWARP; ++w) am = fmaxf(am, red[item & 1][w]);
+        const int e2 = f16_range_exponent(am);
+        inv2e = ldexpf(1.0f, -e2);
+        if (tid == 0) p.scales[((static_cast<size_t>(which) * p.B + b) * H + h) * p.nblk + blk] = ldexpf(1.0f, e2);
+        if (which < 2 && tid < NPAIR) {
+          float m = 0.f;
+#pragma unroll
+          for (int w = 0; w < NWARP; ++w) m = fmaxf(m, pst[item & 1][w][tid]);
+          p.pair_stat[((static_cast<size_t>(which) * p.B * H + b * H + h) * p.nblk + blk) * NPAIR + tid] = m;
+        }
+      }
       uint16_t* dst = static_cast<uint16_t*>(which == 0 ? p.dst[0] : (which == 1 ? p.dst[1] : p.dst[2]));
 #pragma unroll
       for (int i = 0; i < kTokPerThread; ++i) {
@@ -283,10 +306,14 @@ rope_qkv_kernel(const RopeParams p) {
         if constexpr (OUT == kOutF16) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float a = fabsf(x[i][e]);
-            if (a > 65504.f) {
-              range_hit = true;
-              x[i][e] = copysignf(65504.f, x[i][e]);
+            if constexpr (HP) {
+              x[i][e] = __fmul_rn(x[i][e], inv2e);            // exact: a power of two
+            } else {
+              const float a = fabsf(x[i][e]);
+              if (a > 65504.f) {
+                range_hit = true;
+                x[i][e] = copysignf(65504.f, x[i][e]);
+              }
             }
           }
           o.x = pack_f16(x[i][0], x[i][1]); o.y = pack_f16(x[i][2], x[i][3]);
@@ -399,13 +426,13 @@ __global__ void __launch_bounds__(256) repair_gather_kernel(const GatherParams p
   if (p.norm_w != nullptr) {
     float ss = 0.f;
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) ss = fmaf(k[e], k[e], ss);
+    for (int e = 0; e < CPL; ++e) ss = __fmaf_rn(k[e], k[e], ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float rr = __frsqrt_rn(fmaf(ss, 1.0f / D, p.eps));
+    const float rr = norm_factor(ss, D, p.eps);
     const float* w = p.norm_w + (stream * 2 + 1) * D + c0;
 #pragma unroll
-    for (int e = 0; e < CPL; ++e) k[e] = k[e] * rr * w[e];
+    for (int e = 0; e < CPL; ++e) k[e] = norm_scale(k[e], rr, w[e]);
   }
   const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
 #pragma unroll
@@ -414,9 +441,7 @@ __global__ void __launch_bounds__(256) repair_gather_kernel(const GatherParams p
     pair_axis(c0 / 2 + j, n0, n1, n2, axis, ii, n);
     float cs, sn;
     pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs, sn);
-    const float a = k[2 * j], bb = k[2 * j + 1];
-    k[2 * j] = a * cs - bb * sn;
-    k[2 * j + 1] = a * sn + bb * cs;
+    rotate_pair(k[2 * j], k[2 * j + 1], cs, sn, k[2 * j], k[2 * j + 1]);
   }
   bool range_hit = false;
   uint32_t kw[CPL / 2], vw[CPL / 2];
@@ -461,12 +486,19 @@ cudaError_t launch_rope_t(const RopeParams& p, cudaStream_t st) {
   constexpr int NT = D / 8 * kTok / kTokPerThread;
   dim3 grid(p.nblk, p.B);
   const bool repair = OUT == kOutE4M3 && p.score != nullptr;
+  if constexpr (OUT == kOutF16) {
+    if (p.hp) {
+      if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, false, true><<<grid, NT, 0, st>>>(p);
+      else rope_qkv_kernel<D, OUT, false, false, true><<<grid, NT, 0, st>>>(p);
+      return cudaGetLastError();
+    }
+  }
   if (repair) {
-    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, OUT == kOutE4M3><<<grid, NT, 0, st>>>(p);
-    else rope_qkv_kernel<D, OUT, false, OUT == kOutE4M3><<<grid, NT, 0, st>>>(p);
+    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, OUT == kOutE4M3, false><<<grid, NT, 0, st>>>(p);
+    else rope_qkv_kernel<D, OUT, false, OUT == kOutE4M3, false><<<grid, NT, 0, st>>>(p);
   } else {
-    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, false><<<grid, NT, 0, st>>>(p);
-    else rope_qkv_kernel<D, OUT, false, false><<<grid, NT, 0, st>>>(p);
+    if (p.norm_w != nullptr) rope_qkv_kernel<D, OUT, true, false, false><<<grid, NT, 0, st>>>(p);
+    else rope_qkv_kernel<D, OUT, false, false, false><<<grid, NT, 0, st>>>(p);
   }
   return cudaGetLastError();
 }

@@ -10,6 +10,8 @@ Entry points mirror the C names:
   quant_fp8    per-(b, h, 128-token block) e4m3 quantisation
   fwd_bf16     attention forward with 16-bit operands, bf16 output
   fwd_fp8      attention forward with e4m3 operands, bf16 output
+  rope_qkv_hp / fwd_bf16_hp   the high-precision 16-bit path (range scales,
+               split-precision Q.K^T on the outlier channel pairs)
   joint_attention  the whole path in one call (host or device tensors)
 """
 from __future__ import annotations
@@ -36,6 +38,7 @@ _NAME_CODE = {"bf16": BF16, "fp16": FP16, "e4m3": E4M3, "fp8": E4M3}
 SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fwd_fp8_repair",
            "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc",
            "jattn_joint_attention_host", "jattn_joint_attention_host_workspace", "jattn_fwd_bf16", "jattn_fwd_fp8",
+           "jattn_rope_qkv_hp", "jattn_rope_qkv_hp_workspace", "jattn_fwd_bf16_hp",
            "jattn_device_status", "jattn_last_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -78,6 +81,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.jattn_fwd_fp8_repair_noalloc.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, f32, vp, vp,
                                                  vp, f32, vp]
     lib.jattn_fwd_bf16.argtypes = [sp, i32, vp, vp, vp, vp, vp, f32, vp]
+    lib.jattn_rope_qkv_hp.argtypes = [sp, vp, vp, vp, vp, f32, ctypes.POINTER(i32), vp, f32, vp, vp, vp, vp, vp,
+                                      vp, vp, ctypes.c_size_t, vp]
+    lib.jattn_rope_qkv_hp_workspace.argtypes = [sp]
+    lib.jattn_fwd_bf16_hp.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
     lib.jattn_last_device_status.argtypes = [vp]
@@ -89,6 +96,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
         if name not in ("jattn_status_string", "jattn_version"):
             getattr(lib, name).restype = i32
     lib.jattn_fwd_fp8_repair_workspace.restype = ctypes.c_size_t
+    lib.jattn_rope_qkv_hp_workspace.restype = ctypes.c_size_t
     lib.jattn_joint_attention_host_workspace.restype = ctypes.c_size_t
     _lib = lib
     return lib
@@ -293,6 +301,77 @@ def fwd_fp8(q8, k8, v8, scales, o=None, lse=None, want_lse=False, softmax_scale:
     return o, lse
 
 
+CORR_COLS = 16        # columns of one correction row (hi and lo of 8 channels)
+
+
+def rope_qkv_hp(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int], theta: float = 10000.0, out=None,
+                workspace=None, stream=None, norm_w=None, eps: float = 1e-6):
+    """The high-precision 16-bit prologue (jattn_rope_qkv_hp): fp16 q, k, v
+    [B, H, S, d] scaled by powers of two 2^-e per (Q|K|V, b, h, block) --
+    e = 0 unless the block reaches past the fp16 range --, the scales 2^e
+    fp32 [3, B, H, ceil(S/128)], and the correction rows qc, kc fp16
+    [B, H, S, 16] of the 4 channel pairs per (b, h) with the largest
+    max|q_pair| * max|k_pair|.  Returns (q, k, v, scales, qc, kc)."""
+    lib = load()
+    parts = [qkv_txt, qkv_img, qkv_ref]
+    ref = next(t for t in parts if t is not None)
+    B, H, d, lens = _streams(parts)
+    S = sum(lens)
+    dev = ref.device
+    _positions(pos, S, dev)
+    shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
+    need = lib.jattn_rope_qkv_hp_workspace(ctypes.byref(shape))
+    if out is None:
+        q = torch.empty(B, H, S, d, dtype=torch.float16, device=dev)
+        out = (q, torch.empty_like(q), torch.empty_like(q),
+               torch.empty(3, B, H, n_blocks(S), dtype=torch.float32, device=dev),
+               torch.empty(B, H, S, CORR_COLS, dtype=torch.float16, device=dev),
+               torch.empty(B, H, S, CORR_COLS, dtype=torch.float16, device=dev))
+    q, k, v, scales, qc, kc = out
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _dev_shape(t, name, torch.float16, (B, H, S, d))
+    _dev_shape(scales, "scales", torch.float32, (3, B, H, n_blocks(S)))
+    _dev_shape(qc, "qc", torch.float16, (B, H, S, CORR_COLS))
+    _dev_shape(kc, "kc", torch.float16, (B, H, S, CORR_COLS))
+    if norm_w is not None:
+        _dev_shape(norm_w, "norm_w", torch.float32, (3, 2, d))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace must hold at least {need} bytes, got {workspace.numel()}")
+    sp = (ctypes.c_int32 * 3)(*[int(x) for x in split])
+    _check(lib.jattn_rope_qkv_hp(ctypes.byref(shape), _ptr(qkv_txt), _ptr(qkv_img), _ptr(qkv_ref), _ptr(pos),
+                                 float(theta), sp, _ptr(norm_w), float(eps), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(scales), _ptr(qc), _ptr(kc), _ptr(workspace), workspace.numel(),
+                                 _stream(stream)), "jattn_rope_qkv_hp")
+    return q, k, v, scales, qc, kc
+
+
+def rope_qkv_hp_workspace_bytes(B: int, H: int, S_txt: int, S_img: int, S_ref: int, d: int) -> int:
+    return load().jattn_rope_qkv_hp_workspace(ctypes.byref(make_shape(B, H, S_txt, S_img, S_ref, d)))
+
+
+def fwd_bf16_hp(q, k, v, scales, qc, kc, o=None, lse=None, want_lse=False, softmax_scale: float = 0.0,
+                stream=None):
+    """The high-precision 16-bit forward (jattn_fwd_bf16_hp) on the operands
+    rope_qkv_hp wrote."""
+    lib = load()
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, H, S, d], got {tuple(q.shape)}")
+    B, H, S, d = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_shape(t, n, torch.float16, (B, H, S, d))
+    _dev_shape(scales, "scales", torch.float32, (3, B, H, n_blocks(S)))
+    _dev_shape(qc, "qc", torch.float16, (B, H, S, CORR_COLS))
+    _dev_shape(kc, "kc", torch.float16, (B, H, S, CORR_COLS))
+    o, lse = _fwd_outputs(B, H, S, d, q.device, o, lse, want_lse)
+    shape = make_shape(B, H, S, 0, 0, d)
+    _check(lib.jattn_fwd_bf16_hp(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(scales), _ptr(qc), _ptr(kc),
+                                 _ptr(o), _ptr(lse), float(softmax_scale), _stream(stream)), "jattn_fwd_bf16_hp")
+    return o, lse
+
+
 def device_status(clear: bool = True, stream=None):
     """(status code, raw bits) of the current device's status word."""
     lib = load()
@@ -402,9 +481,11 @@ def fwd_fp8_repair_noalloc(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int],
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
                     operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None,
-                    norm_w=None, eps: float = 1e-6, workspace=None):
+                    norm_w=None, eps: float = 1e-6, workspace=None, precise: bool = False):
     """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8),
-    with the query/key RMSNorm fused into rope_qkv when ``norm_w`` is given.
+    with the query/key RMSNorm fused into rope_qkv when ``norm_w`` is given;
+    ``precise`` (device tensors, BF16 path) selects the high-precision pair
+    rope_qkv_hp -> fwd_bf16_hp.
 
     CUDA tensors: the device entry points, asynchronous on ``stream``.
     CPU tensors (pinned for overlap): jattn_joint_attention_host, which
@@ -445,7 +526,10 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
                                               ctypes.c_void_p(st.cuda_stream)), "jattn_joint_attention_host")
         st.synchronize()
         return out
-    if path == "bf16":
+    if path == "bf16" and precise:
+        q, k, v, sc, qc, kc = rope_qkv_hp(*parts, pos, split, theta, stream=stream, norm_w=norm_w, eps=eps)
+        o, lse = fwd_bf16_hp(q, k, v, sc, qc, kc, want_lse=want_lse, stream=stream)
+    elif path == "bf16":
         q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream, norm_w=norm_w, eps=eps)
         o, lse = fwd_bf16(q, k, v, want_lse=want_lse, stream=stream)
     elif path == "fp8":

@@ -162,6 +162,53 @@ jattn_status jattn_fwd_fp8(const jattn_shape* shape, const void* q8, const void*
                            float softmax_scale, void* stream);
 
 /*
+ * High-precision 16-bit path: the BF16 path of jattn_rope_qkv(_norm) +
+ * jattn_fwd_bf16, computed so that it stays within the BF16 path's error
+ * bars (rel-L2 5e-3, max-abs 2e-2 against the exact result) also when a few
+ * channels of a head carry activation outliers, and with no saturation.
+ * ("Speed Up Image Generation with FLUX 3 Image Klein on NVIDIA Blackwell
+ * GPUs", section "Quantized and sparse attention": dense BF16 attention is
+ * the accuracy reference of the quantised variants.)  Two differences from
+ * the plain fp16-operand path:
+ *   - range: every (Q|K|V, batch, head, 128-token block) tile is stored as
+ *     fp16(x * 2^-e), e >= 0 the smallest exponent that keeps the tile
+ *     within +-65504 (0 for all ordinary inputs); the scales 2^e are folded
+ *     into the softmax exactly like the e4m3 block scales;
+ *   - precision: fp16 rounding of the rotated Q / K costs each logit an
+ *     error proportional to |q_pair| |k_pair| summed over channel pairs; per
+ *     (batch, head) the 4 pairs with the largest max|q_pair| * max|k_pair|
+ *     (ties to the lower pair) get their rounding residual back: correction
+ *     rows qc = [hi | lo] and kc = [lo | hi] of those 8 channels (hi the
+ *     stored fp16 value, lo = fp16(x - hi)) add hi_q lo_k + lo_q hi_k to
+ *     every logit through one more 16-deep MMA.
+ *
+ * jattn_rope_qkv_hp: the prologue (assembly, optional query/key RMSNorm as
+ * jattn_rope_qkv_norm -- norm_w may be NULL for none --, RoPE) and the
+ * correction rows, three launches on `stream`.
+ *   qkv_*, pos, theta, split, norm_w, eps : as jattn_rope_qkv_norm.
+ *   q, k, v    : fp16 [B, H, S, d], the scaled values fp16(x * 2^-e).
+ *   scales     : fp32 [3][B][H][ceil(S/128)], the powers of two 2^e (Q, K, V).
+ *   qc, kc     : fp16 [B, H, S, 16], the correction rows.
+ *   workspace  : device scratch of at least jattn_rope_qkv_hp_workspace(shape)
+ *                bytes, 256-byte aligned, owned by the caller (per-block
+ *                pair statistics, the selection, RMSNorm row factors).
+ * jattn_fwd_bf16_hp: the forward on those operands; o, lse, softmax_scale as
+ * jattn_fwd_bf16.
+ * Errors: as jattn_rope_qkv / jattn_fwd_bf16; JATTN_ERR_INVALID_ARG for a
+ * NULL scales, qc, kc or workspace, or a workspace that is too small;
+ * JATTN_ERR_ALIGNMENT for a workspace not 256-byte aligned.
+ */
+size_t jattn_rope_qkv_hp_workspace(const jattn_shape* shape);   /* 0 on invalid arguments */
+jattn_status jattn_rope_qkv_hp(const jattn_shape* shape, const void* qkv_txt, const void* qkv_img,
+                               const void* qkv_ref, const int32_t* pos, float theta,
+                               const int32_t split[3], const float* norm_w, float eps, void* q, void* k,
+                               void* v, float* scales, void* qc, void* kc, void* workspace,
+                               size_t workspace_bytes, void* stream);
+jattn_status jattn_fwd_bf16_hp(const jattn_shape* shape, const void* q, const void* k, const void* v,
+                               const float* scales, const void* qc, const void* kc, void* o, float* lse,
+                               float softmax_scale, void* stream);
+
+/*
  * FP8 attention with token repair ("Speed Up Image Generation with FLUX 3
  * Image Klein on NVIDIA Blackwell GPUs", section "Quantized and sparse
  * attention": a repair budget rho -- 0.005 in the tested configuration --

@@ -211,3 +211,38 @@ def test_last_device_status_is_exported():
     lib = jattn.load()
     assert hasattr(lib, "jattn_last_device_status")
     assert "jattn_last_device_status" in declared_symbols()
+
+
+def test_hp_entry_points_reject_bad_arguments():
+    """jattn_rope_qkv_hp / jattn_fwd_bf16_hp: scales, correction rows and
+    workspace are required; the workspace must be large enough and 256-byte
+    aligned; the shared prologue and forward checks still apply."""
+    lib = jattn.load()
+    sp = _split(16, 56, 56)
+    need = lib.jattn_rope_qkv_hp_workspace(shape(B=2, St=300))
+    assert need > 0 and need % 256 == 0
+    assert lib.jattn_rope_qkv_hp_workspace(shape(d=96)) == 0
+    f = lib.jattn_rope_qkv_hp
+    ok = dict(sh=shape(), sc=A, qc=A, kc=A, ws=A, n=lib.jattn_rope_qkv_hp_workspace(shape()), split=sp, norm=None,
+              eps=1e-6)
+
+    def call(**kw):
+        a = dict(ok, **kw)
+        return f(a["sh"], A, None, None, A, 1e4, a["split"], a["norm"], a["eps"], A, A, A, a["sc"], a["qc"], a["kc"],
+                 a["ws"], a["n"], None)
+    assert call(sc=None) == jattn.ERR_INVALID_ARG
+    assert call(qc=None) == jattn.ERR_INVALID_ARG
+    assert call(kc=None) == jattn.ERR_INVALID_ARG
+    assert call(ws=None) == jattn.ERR_INVALID_ARG
+    assert call(n=ok["n"] - 1) == jattn.ERR_INVALID_ARG
+    assert call(ws=A + 16) == jattn.ERR_ALIGNMENT
+    assert call(qc=A + 8) == jattn.ERR_ALIGNMENT
+    assert call(norm=A, eps=0.0) == jattn.ERR_INVALID_ARG
+    assert call(split=_split(16, 56, 58)) == jattn.ERR_INVALID_ARG
+    assert call(sh=shape(d=96)) == jattn.ERR_UNSUPPORTED
+    g = lib.jattn_fwd_bf16_hp
+    assert g(shape(), A, A, A, None, A, A, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
+    assert g(shape(), A, A, A, A, None, A, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
+    assert g(shape(), A, A, A, A, A, A + 8, A, None, 0.0, None) == jattn.ERR_ALIGNMENT
+    assert g(shape(), None, A, A, A, A, A, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
+    assert g(shape(d=96), A, A, A, A, A, A, A, None, 0.0, None) == jattn.ERR_UNSUPPORTED
