@@ -11,7 +11,8 @@
 //   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one thread
 //               per query row (= TMEM lane), online softmax with a lazy
 //               rescale (O and l are rescaled only when the running max grows
-//               by more than 2^8), P written back into the tile's S columns;
+//               by more than 2^15 -- 2^8 with e4m3 P), P written back into
+//               the tile's S columns;
 //               epilogue O / l -> bf16 [B, S, H, d].
 //   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T, O_t += P_t V_j.
 //               Issue order PV_0(j), QK_0(j+1), PV_1(j), QK_1(j+1): each
@@ -49,7 +50,12 @@ constexpr uint32_t kRegsSoftmax = 224;
 constexpr uint32_t kRegsOther = 56;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;   // log2 units: P <= 2^8 before a rescale
+// Lazy rescale: O and l are rescaled only when a row's running max grows by
+// more than this many log2 units, so P <= 2^threshold in between.  16-bit P
+// has room for 2^15 (fewer rescales); e4m3 P keeps 2^8 so that P * 448 / 2^8
+// stays in range without pushing small probabilities into subnormals.
+constexpr float kRescaleThreshold16 = 15.0f;
+constexpr float kRescaleThreshold8 = 8.0f;
 
 __host__ __device__ constexpr uint32_t col_s(int t) { return static_cast<uint32_t>(t) * 128u; }
 __host__ __device__ constexpr uint32_t col_o(int t) { return 256u + static_cast<uint32_t>(t) * 128u; }
@@ -364,7 +370,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
     // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
     // exceeds the e4m3 range while p <= 2^8.  HP: as p * (s_v,j / max s_v)
-    // (powers of two; at most 2^8 in fp16).
+    // (powers of two; at most 2^15 in fp16).
+    constexpr float kRescaleThreshold = FP8 ? kRescaleThreshold8 : kRescaleThreshold16;
     const float p8_log2 = FP8 ? 8.8073549220576042f - kRescaleThreshold : 0.f;   // log2(448) - 8
     // The K / V block scales of the next tile are fetched one tile ahead so
     // that their load latency stays off the S -> P chain.

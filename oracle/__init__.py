@@ -18,6 +18,9 @@ from .joint_attention import (  # noqa: F401
 from .repair import (  # noqa: F401
     repair_count, repair_scores, repair_select, repaired_attention_rows, repaired_attention,
 )
+from .block_sparse import (  # noqa: F401
+    block_means, block_shares, block_select, block_sparse_attention_rows, block_sparse_attention,
+)
 from .fp8 import (  # noqa: F401
     E4M3_MAX, e4m3_decode, e4m3_encode, block_scales, quantize_blocks,
     dequantize_blocks, rounding_ambiguous,
