@@ -61,6 +61,7 @@ def parse(argv=None):
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the FP8-with-repair, query/key-norm prologue and other-workload measurements")
     ap.add_argument("--rho", type=float, default=0.005, help="token-repair budget of the FP8-with-repair block")
+    ap.add_argument("--tau", type=float, default=1.0, help="sparsity of the block-sparse block (0 = dense)")
     return ap.parse_args(argv)
 
 
@@ -354,6 +355,7 @@ def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops, ms_fp8):
     * the prologue with the query/key RMSNorm fused in, against the same
       prologue without it."""
     out = {"fp8_repair": measure_repair(jattn, ctx, w, dinp, args.rho, args.steps, args.warmup, ms_fp8)}
+    out["block_sparse"] = measure_block_sparse(jattn, ctx, w, dinp, args.tau, args.steps, args.warmup)
     B, H, S, d = w.B, w.H, w.S, w.d
     q = torch.empty(B, H, S, d, dtype=torch.float16, device=ctx.dev)
     bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
@@ -369,6 +371,43 @@ def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops, ms_fp8):
                                "achieved_GBps": round(nbytes / res["qk_norm"] / 1e6, 1),
                                "note": "fp16 output; back-to-back calls (no flush between them)"}
     return out
+
+
+def measure_block_sparse(jattn, ctx: Ctx, w, dinp, tau, steps, warmup):
+    """Block-sparse forward at tau on the fp16 operands of the prologue: the
+    call (block means, selection, sparse forward) timed alone; TFLOPS on the
+    dense FLOP count (the work the call stands in for) and on the kept
+    blocks' own FLOPs."""
+    B, H, S, d = w.B, w.H, w.S, w.d
+    q, k, v, _ = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                                "fp16")
+    o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=ctx.dev)
+    ws = torch.empty(jattn.load().jattn_fwd_block_sparse_workspace(
+        jattn.ctypes.byref(jattn.make_shape(B, H, S, 0, 0, d))), dtype=torch.uint8, device=ctx.dev)
+    _, kl, kc = jattn.fwd_block_sparse(q, k, v, tau, o=o, want_blocks=True, workspace=ws)
+    ms, _ = time_calls(ctx, lambda ev: jattn.fwd_block_sparse(q, k, v, tau, o=o, workspace=ws, stream=ctx.stream),
+                       steps, warmup)
+    code, bits = jattn.device_status(clear=True)
+    if code != jattn.OK:
+        raise RuntimeError(f"device status {code} bits {bits} after the block-sparse run")
+    # FLOPs of the kept (query tile, key tile) pairs: each 256-row block of
+    # full query rows times the kept keys (tails counted at their length)
+    n_qb, n_kb = kc.shape[-1], jattn.n_blocks(S)
+    klen = torch.full((n_kb,), 128, dtype=torch.float64)
+    klen[-1] = S - 128 * (n_kb - 1)
+    qlen = torch.full((n_qb,), 256, dtype=torch.float64)
+    qlen[-1] = S - 256 * (n_qb - 1)
+    kept_keys = torch.zeros(B, H, n_qb, dtype=torch.float64)
+    kl, kc = kl.cpu(), kc.cpu()
+    for b in range(B):
+        for h in range(H):
+            for i in range(n_qb):
+                kept_keys[b, h, i] = klen[kl[b, h, i, :kc[b, h, i]].long()].sum()
+    kept_flops = float(4 * d * (kept_keys * qlen).sum())
+    return {"tau": tau, "ms": round(ms, 4), "kept_fraction": round(kept_flops / w.flops, 4),
+            "dense_equivalent_tflops": round(w.flops / ms / 1e9, 2),
+            "kept_tflops": round(kept_flops / ms / 1e9, 2), "gpu_launches_per_call": 3,
+            "operands": "fp16 from jattn_rope_qkv (prologue not timed)"}
 
 
 def measure_repair(jattn, ctx: Ctx, w, dinp, rho, steps, warmup, ms_fp8):

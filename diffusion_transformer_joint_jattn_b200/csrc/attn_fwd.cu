@@ -179,7 +179,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int qp = blockIdx.x;                           // pair of query tiles
   const int bh = blockIdx.y;
   const int b = bh / p.H, h = bh % p.H;
-  const int n_kv = p.n_kv;
+  // Key tiles this CTA walks: all n_kv in order, or (block-sparse) the
+  // first kv_count entries of its kv_list row.
+  const int32_t* kv_list = p.kv_list != nullptr
+                               ? p.kv_list + (static_cast<size_t>(bh) * gridDim.x + qp) * p.n_kv
+                               : nullptr;
+  const int n_kv = kv_list != nullptr ? p.kv_count[static_cast<size_t>(bh) * gridDim.x + qp] : p.n_kv;
+  auto kv_tile = [&](int j) { return kv_list != nullptr ? __ldg(kv_list + j) : j; };
 
   if (threadIdx.x == 0) {
     mbar_init(&bar->q_full, 1);
@@ -235,15 +241,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         const int ks = j % C::KS;
         if (!mbar_wait(&bar->k_empty[ks], ((j / C::KS) & 1) ^ 1, ctl)) break;
         mbar_arrive_expect_tx(&bar->k_full[ks], C::TB + C::CT);
+        const int kt = kv_tile(j);
         for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
-        if constexpr (HP) tma_load_3d(&tmKc, &bar->k_full[ks], sKc + ks * C::CT, 0, j * BN, bh);
+          tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
+        if constexpr (HP) tma_load_3d(&tmKc, &bar->k_full[ks], sKc + ks * C::CT, 0, kt * BN, bh);
         nk = j + 1;
         const int vs = j % C::VS;
         if (!mbar_wait(&bar->v_empty[vs], ((j / C::VS) & 1) ^ 1, ctl)) break;
         mbar_arrive_expect_tx(&bar->v_full[vs], C::TB);
         for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmV, &bar->v_full[vs], sV + vs * C::TB + x * C::BOXB, x * C::BOX_ELEMS, j * BN, bh);
+          tma_load_3d(&tmV, &bar->v_full[vs], sV + vs * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
         nv = j + 1;
       }
       // Drain: every load issued must have landed before the CTA may exit.
@@ -363,7 +370,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       sc_k = p.scales + plane + bhn;
       sc_v = p.scales + 2 * plane + bhn;
       float mv = 0.f;
-      for (int j = lane; j < n_kv; j += 32) mv = fmaxf(mv, sc_v[j]);
+      for (int j = lane; j < p.n_kv; j += 32) mv = fmaxf(mv, sc_v[j]);   // every tile: ratios stay <= 1
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
       max_sv = mv > 0.f ? mv : 1.f;
@@ -376,24 +383,27 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     // The K / V block scales of the next tile are fetched one tile ahead so
     // that their load latency stays off the S -> P chain.
     float sk_nxt = 0.f, sv_nxt = 0.f;
+    int kt_cur = n_kv > 0 ? kv_tile(0) : 0;            // key tile of step j
     if constexpr (SCALED) {
-      sk_nxt = sc_k[0];
-      sv_nxt = sc_v[0];
+      sk_nxt = sc_k[kt_cur];
+      sv_nxt = sc_v[kt_cur];
     }
 
     for (int j = 0; j < n_kv; ++j) {
+      const int kt = kt_cur;
+      if (j + 1 < n_kv) kt_cur = kv_tile(j + 1);
       float c_j = sl2, bias = 0.f;
       if constexpr (SCALED) {
         c_j = sl2 * sq * sk_nxt;
         bias = __log2f(sv_nxt / max_sv) + p8_log2;
         if (j + 1 < n_kv) {
-          sk_nxt = sc_k[j + 1];
-          sv_nxt = sc_v[j + 1];
+          sk_nxt = sc_k[kt_cur];
+          sv_nxt = sc_v[kt_cur];
         }
       }
       // Keys left out of this pass (same for every row of the tile).
       uint4 km = make_uint4(0u, 0u, 0u, 0u);
-      if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * n_kv + j);
+      if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * p.n_kv + kt);
       ok = warp_wait(&bar->s_full[t], j & 1, ctl);
       if (!ok) break;
       __syncwarp();
@@ -406,7 +416,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < BN; ++e) v[e] = __uint_as_float(r[e]);
       }
 
-      const int valid = p.S_kv - j * BN;
+      const int valid = p.S_kv - kt * BN;
       if (valid < BN) {
 #pragma unroll
         for (int e = 0; e < BN; ++e)

@@ -429,6 +429,79 @@ jattn_status jattn_fwd_bf16_hp(const jattn_shape* shape, const void* q, const vo
              : JATTN_ERR_CUDA;
 }
 
+// ---------------------------------------------------------------- block-sparse attention
+
+namespace {
+
+struct SparseLayout {
+  size_t pool, list, count, total;
+};
+
+SparseLayout sparse_layout(const jattn_shape* shape) {
+  const size_t BH = static_cast<size_t>(shape->B) * shape->H;
+  const int S = total_S(shape);
+  const size_t nb = n_blocks(S), nq = (S + 2 * JATTN_BLOCK - 1) / (2 * JATTN_BLOCK), d = shape->d;
+  SparseLayout L{};
+  size_t off = 0;
+  auto seg = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
+  L.pool = seg(2 * BH * nb * d * 4);
+  L.list = seg(BH * nq * nb * 4);
+  L.count = seg(BH * nq * 4);
+  L.total = off;
+  return L;
+}
+
+}  // namespace
+
+size_t jattn_fwd_block_sparse_workspace(const jattn_shape* shape) {
+  if (check_shape(shape) != JATTN_OK) return 0;
+  return sparse_layout(shape).total;
+}
+
+jattn_status jattn_fwd_block_sparse(const jattn_shape* shape, jattn_dtype in_dtype, const void* q, const void* k,
+                                    const void* v, float tau, void* workspace, size_t workspace_bytes, void* o,
+                                    float* lse, int32_t* kv_list, int32_t* kv_count, float softmax_scale,
+                                    void* stream) {
+  if (in_dtype != JATTN_BF16 && in_dtype != JATTN_FP16) return JATTN_ERR_UNSUPPORTED;
+  if (!(tau >= 0.f) || !std::isfinite(tau)) return JATTN_ERR_INVALID_ARG;
+  jattn_status st = check_shape(shape);
+  if (st != JATTN_OK) return st;
+  const SparseLayout L = sparse_layout(shape);
+  if (workspace == nullptr || workspace_bytes < L.total) return JATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return JATTN_ERR_ALIGNMENT;
+  if ((kv_list != nullptr && (reinterpret_cast<uintptr_t>(kv_list) & 3u)) ||
+      (kv_count != nullptr && (reinterpret_cast<uintptr_t>(kv_count) & 3u)))
+    return JATTN_ERR_ALIGNMENT;
+  jattn::FwdParams p{};
+  if ((st = fwd_common(shape, q, k, v, o, lse, softmax_scale, p)) != JATTN_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  jattn::SparseParams sp{};
+  sp.q = q;
+  sp.k = k;
+  sp.BH = p.B * p.H;
+  sp.S = p.S;
+  sp.d = shape->d;
+  sp.nblk = p.n_kv;
+  sp.n_qb = (p.n_tiles + 1) / 2;
+  sp.scale = p.scale_log2 / 1.4426950408889634f;
+  sp.tau = tau;
+  sp.pool = reinterpret_cast<float*>(ws + L.pool);
+  sp.kv_list = kv_list != nullptr ? kv_list : reinterpret_cast<int32_t*>(ws + L.list);
+  sp.kv_count = kv_count != nullptr ? kv_count : reinterpret_cast<int32_t*>(ws + L.count);
+  if (jattn::launch_block_select(sp, in_dtype == JATTN_BF16, cs) != cudaSuccess) return JATTN_ERR_CUDA;
+  p.kv_list = sp.kv_list;
+  p.kv_count = sp.kv_count;
+  CUtensorMap tq, tk, tv;
+  const int BH = p.B * p.H;
+  const int kv_rows = jattn::fwd_kv_rows();
+  if ((st = make_map(&tq, q, BH, p.S, shape->d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
+  if ((st = make_map(&tk, k, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
+  if ((st = make_map(&tv, v, BH, p.S, shape->d, 2, kv_rows)) != JATTN_OK) return st;
+  return jattn::launch_fwd_f16(p, shape->d, in_dtype == JATTN_BF16, tq, tk, tv, cs) == cudaSuccess ? JATTN_OK
+                                                                                                  : JATTN_ERR_CUDA;
+}
+
 // ---------------------------------------------------------------- FP8 with token repair
 
 int32_t jattn_repair_count(const jattn_shape* shape, float rho) {

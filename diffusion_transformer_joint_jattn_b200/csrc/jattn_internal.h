@@ -79,6 +79,21 @@ struct CorrParams {
 
 cudaError_t launch_qk_correction(const CorrParams& p, cudaStream_t st);
 
+// Block-sparse attention: selection of the key tiles each 256-row query
+// block attends to.
+struct SparseParams {
+  const void* q;                // [B*H][S][d] 16-bit (rotated)
+  const void* k;
+  int BH, S, d, nblk, n_qb;     // nblk = ceil(S / 128) key tiles, n_qb = ceil(S / 256) query blocks
+  float scale;                  // softmax scale
+  float tau;                    // keep a key block iff its estimated share >= tau / nblk
+  float* pool;                  // [2][B*H][nblk][d] column sums of every 128-token tile of Q, K
+  int32_t* kv_list;             // [B*H][n_qb][nblk] kept key tiles, ascending (first kv_count entries)
+  int32_t* kv_count;            // [B*H][n_qb]
+};
+
+cudaError_t launch_block_select(const SparseParams& p, bool in_bf16, cudaStream_t st);
+
 struct QuantParams {
   const void* x;                // [BH, S, d] 16-bit
   void* x8;                     // [BH, S, d] e4m3
@@ -96,6 +111,8 @@ struct FwdParams {
   const uint32_t* kmask;        // null, or [B*H][n_kv][4] words: bit set = key left out of this pass
   const float* lse_prev;        // null, or [B, H, S]: o already holds a partial result with this
                                 // LSE over other keys; the pass merges its own into o (and lse)
+  const int32_t* kv_list;       // null, or [B*H][gridDim.x][n_kv]: the key tiles each CTA (pair of
+  const int32_t* kv_count;      //   query tiles) walks, ascending, and how many ([B*H][gridDim.x])
   uint32_t* status;
   uint64_t timeout_ns;
   long long* trace;             // development timing probe; always null in the library

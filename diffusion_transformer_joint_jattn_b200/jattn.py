@@ -39,6 +39,7 @@ SYMBOLS = ("jattn_rope_qkv", "jattn_rope_qkv_norm", "jattn_quant_fp8", "jattn_fw
            "jattn_fwd_fp8_repair_workspace", "jattn_repair_count", "jattn_fwd_fp8_repair_noalloc",
            "jattn_joint_attention_host", "jattn_joint_attention_host_workspace", "jattn_fwd_bf16", "jattn_fwd_fp8",
            "jattn_rope_qkv_hp", "jattn_rope_qkv_hp_workspace", "jattn_fwd_bf16_hp",
+           "jattn_fwd_block_sparse", "jattn_fwd_block_sparse_workspace",
            "jattn_device_status", "jattn_last_device_status", "jattn_selftest_wait_timeout", "jattn_status_string",
            "jattn_version")
 
@@ -85,6 +86,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                                       vp, vp, ctypes.c_size_t, vp]
     lib.jattn_rope_qkv_hp_workspace.argtypes = [sp]
     lib.jattn_fwd_bf16_hp.argtypes = [sp, vp, vp, vp, vp, vp, vp, vp, vp, f32, vp]
+    lib.jattn_fwd_block_sparse.argtypes = [sp, i32, vp, vp, vp, f32, vp, ctypes.c_size_t, vp, vp, vp, vp, f32, vp]
+    lib.jattn_fwd_block_sparse_workspace.argtypes = [sp]
     lib.jattn_fwd_fp8.argtypes = [sp, vp, vp, vp, vp, vp, vp, f32, vp]
     lib.jattn_device_status.argtypes = [vp, i32, ctypes.POINTER(ctypes.c_uint32)]
     lib.jattn_last_device_status.argtypes = [vp]
@@ -97,6 +100,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
             getattr(lib, name).restype = i32
     lib.jattn_fwd_fp8_repair_workspace.restype = ctypes.c_size_t
     lib.jattn_rope_qkv_hp_workspace.restype = ctypes.c_size_t
+    lib.jattn_fwd_block_sparse_workspace.restype = ctypes.c_size_t
     lib.jattn_joint_attention_host_workspace.restype = ctypes.c_size_t
     _lib = lib
     return lib
@@ -370,6 +374,44 @@ def fwd_bf16_hp(q, k, v, scales, qc, kc, o=None, lse=None, want_lse=False, softm
     _check(lib.jattn_fwd_bf16_hp(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(scales), _ptr(qc), _ptr(kc),
                                  _ptr(o), _ptr(lse), float(softmax_scale), _stream(stream)), "jattn_fwd_bf16_hp")
     return o, lse
+
+
+def fwd_block_sparse(q, k, v, tau: float, o=None, lse=None, want_lse: bool = False, want_blocks: bool = False,
+                     workspace=None, softmax_scale: float = 0.0, stream=None):
+    """Block-sparse attention forward (jattn_fwd_block_sparse) on fp16/bf16
+    [B, H, S, d] operands: per 256-row query block, only the 128-key blocks
+    whose estimated attention share reaches tau / n_kb (and the largest).
+    Returns o (and lse; and, with want_blocks, kv_list int32 [B, H, n_qb,
+    n_kb] and kv_count int32 [B, H, n_qb])."""
+    lib = load()
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, H, S, d], got {tuple(q.shape)}")
+    B, H, S, d = q.shape
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _dev_shape(t, n, q.dtype, (B, H, S, d))
+    o, lse = _fwd_outputs(B, H, S, d, q.device, o, lse, want_lse)
+    shape = make_shape(B, H, S, 0, 0, d)
+    need = lib.jattn_fwd_block_sparse_workspace(ctypes.byref(shape))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _dev(workspace, "workspace", torch.uint8)
+    if workspace.numel() < need:
+        raise ValueError(f"workspace must hold at least {need} bytes, got {workspace.numel()}")
+    n_qb, n_kb = -(-S // (2 * BLOCK)), n_blocks(S)
+    kv_list = kv_count = None
+    if want_blocks:
+        kv_list = torch.empty(B, H, n_qb, n_kb, dtype=torch.int32, device=q.device)
+        kv_count = torch.empty(B, H, n_qb, dtype=torch.int32, device=q.device)
+    _check(lib.jattn_fwd_block_sparse(ctypes.byref(shape), _DTYPE_CODE[q.dtype], _ptr(q), _ptr(k), _ptr(v),
+                                      float(tau), _ptr(workspace), workspace.numel(), _ptr(o), _ptr(lse),
+                                      _ptr(kv_list), _ptr(kv_count), float(softmax_scale), _stream(stream)),
+           "jattn_fwd_block_sparse")
+    out = [o]
+    if want_lse:
+        out.append(lse)
+    if want_blocks:
+        out += [kv_list, kv_count]
+    return out[0] if len(out) == 1 else tuple(out)
 
 
 def device_status(clear: bool = True, stream=None):

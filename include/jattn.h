@@ -209,6 +209,44 @@ jattn_status jattn_fwd_bf16_hp(const jattn_shape* shape, const void* q, const vo
                                float softmax_scale, void* stream);
 
 /*
+ * Block-sparse attention forward, 16-bit operands ("Speed Up Image Generation
+ * with FLUX 3 Image Klein on NVIDIA Blackwell GPUs", sections "Quantized and
+ * sparse attention" and "Optimized single-GPU deployment": Sol-Attention, a
+ * block-sparse attention whose sparsity tau controls -- higher tau drops
+ * more blocks -- run dense until a noise-level cutoff, which is the caller's
+ * choice of tau = 0 for those steps).  The page names no selection rule;
+ * this library reads it as:
+ *   - queries in blocks of 256 joint tokens, keys in blocks of 128 (the last
+ *     block of each may be shorter), each block represented by the mean of
+ *     its rotated rows;
+ *   - the estimated attention share of key block J for query block I is the
+ *     softmax over J of qbar_I . kbar_J * softmax_scale;
+ *   - J is kept iff its share >= tau / n_kb (n_kb = ceil(S/128): tau times a
+ *     uniform share), and the largest share is always kept (ties to the
+ *     lower J); tau = 0 keeps everything (the dense result);
+ *   - every query row attends, with an exact softmax, to the keys of its
+ *     block's kept key blocks only.
+ * Three launches on `stream`: block means, selection, the forward walking
+ * the kept key tiles.
+ *   q, k, v, in_dtype, o, lse, softmax_scale : as jattn_fwd_bf16.
+ *   tau        : >= 0 and finite, else JATTN_ERR_INVALID_ARG.
+ *   workspace  : device scratch of at least
+ *                jattn_fwd_block_sparse_workspace(shape) bytes, 256-byte
+ *                aligned, owned by the caller.
+ *   kv_list    : NULL, or int32 [B][H][ceil(S/256)][ceil(S/128)]: row (b, h,
+ *                I) receives the kept key blocks of query block I in
+ *                ascending order (the entries past its count are undefined);
+ *   kv_count   : NULL, or int32 [B][H][ceil(S/256)]: how many.
+ * Errors: as jattn_fwd_bf16; JATTN_ERR_INVALID_ARG for a NULL or too small
+ * workspace; JATTN_ERR_ALIGNMENT for a workspace not 256-byte aligned.
+ */
+size_t jattn_fwd_block_sparse_workspace(const jattn_shape* shape);   /* 0 on invalid arguments */
+jattn_status jattn_fwd_block_sparse(const jattn_shape* shape, jattn_dtype in_dtype, const void* q, const void* k,
+                                    const void* v, float tau, void* workspace, size_t workspace_bytes, void* o,
+                                    float* lse, int32_t* kv_list, int32_t* kv_count, float softmax_scale,
+                                    void* stream);
+
+/*
  * FP8 attention with token repair ("Speed Up Image Generation with FLUX 3
  * Image Klein on NVIDIA Blackwell GPUs", section "Quantized and sparse
  * attention": a repair budget rho -- 0.005 in the tested configuration --

@@ -246,3 +246,25 @@ def test_hp_entry_points_reject_bad_arguments():
     assert g(shape(), A, A, A, A, A, A + 8, A, None, 0.0, None) == jattn.ERR_ALIGNMENT
     assert g(shape(), None, A, A, A, A, A, A, None, 0.0, None) == jattn.ERR_INVALID_ARG
     assert g(shape(d=96), A, A, A, A, A, A, A, None, 0.0, None) == jattn.ERR_UNSUPPORTED
+
+
+def test_block_sparse_rejects_bad_arguments():
+    lib = jattn.load()
+    need = lib.jattn_fwd_block_sparse_workspace(shape(St=300))
+    assert need > 0 and need % 256 == 0
+    assert lib.jattn_fwd_block_sparse_workspace(shape(d=96)) == 0
+    f = lib.jattn_fwd_block_sparse
+    n = lib.jattn_fwd_block_sparse_workspace(shape())
+
+    def call(dt=jattn.FP16, tau=1.0, ws=A, nb=n, o=A, kl=None, kc=None, sh=None):
+        return f(sh or shape(), dt, A, A, A, tau, ws, nb, o, None, kl, kc, 0.0, None)
+    assert call(dt=jattn.E4M3) == jattn.ERR_UNSUPPORTED
+    assert call(tau=-1.0) == jattn.ERR_INVALID_ARG
+    assert call(tau=float("nan")) == jattn.ERR_INVALID_ARG
+    assert call(tau=float("inf")) == jattn.ERR_INVALID_ARG
+    assert call(ws=None) == jattn.ERR_INVALID_ARG
+    assert call(nb=n - 1) == jattn.ERR_INVALID_ARG
+    assert call(ws=A + 16) == jattn.ERR_ALIGNMENT
+    assert call(o=None) == jattn.ERR_INVALID_ARG
+    assert call(kl=A + 2) == jattn.ERR_ALIGNMENT
+    assert call(sh=shape(d=96)) == jattn.ERR_UNSUPPORTED
