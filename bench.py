@@ -1,8 +1,10 @@
 """Benchmark: joint-attention TFLOPS on the 2048x2048 Base T2I workload.
 
-One step = one pass of the whole hot path over one batch: jattn_rope_qkv
-(joint-sequence assembly + 2D axial RoPE) followed by jattn_fwd_bf16 (or the
-e4m3 pair for the FP8 path).  TFLOPS = 4 * B * H * S^2 * d / step time.
+One step = one pass of the whole hot path over one batch: jattn_rope_qkv_hp
+(joint-sequence assembly + 2D axial RoPE, range scales, correction rows)
+followed by jattn_fwd_bf16_hp -- the BF16 path that meets the BF16 error bars
+--, with the plain fp16-operand pair, the e4m3 pair and the next-row paths
+reported beside it.  TFLOPS = 4 * B * H * S^2 * d / step time.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -285,16 +287,21 @@ def run_ours(args, rank, world, local):
     peaks, peak_src = load_peaks()
     full = args.workload == WORKLOAD
 
+    # The headline BF16 path is the high-precision one (range scales and
+    # split-precision Q.K^T): the one that meets the BF16 error bars on every
+    # workload.  The plain fp16-operand path is reported beside it.
     sampler = ClockSampler(local)
     sampler.start()
-    ms, pro_ms, fwd_ms, fwd_med, fwd_min = measure_path(jattn, ctx, w, dinp, "bf16", args.steps, args.warmup)
+    ms, pro_ms, fwd_ms, fwd_med, fwd_min = measure_path(jattn, ctx, w, dinp, "bf16_hp", args.steps, args.warmup)
     clocks = sampler.stop()
-    msh, proh, fwdh, fwdh_med, fwdh_min = measure_path(jattn, ctx, w, dinp, "bf16_hp", args.steps, args.warmup)
-    hp = {"value": round(whole_job_tflops(flops, msh), 2), "unit": UNIT, "ms_per_step": round(msh, 4),
-          "prologue_ms": round(proh, 4), "fwd_ms": round(fwdh, 4), "fwd_ms_median": round(fwdh_med, 4),
-          "fwd_ms_min": round(fwdh_min, 4), "gpu_launches_per_step": 4,
-          "roofline": tensor_roofline(flops, fwdh, peaks, peak_src, False, None,
-                                      "attn_fwd_kernel<128, fp16 operands, high precision>")}
+    msf, prof, fwdf, fwdf_med, fwdf_min = measure_path(jattn, ctx, w, dinp, "bf16", args.steps, args.warmup)
+    fast = {"value": round(whole_job_tflops(flops, msf), 2), "unit": UNIT, "ms_per_step": round(msf, 4),
+            "prologue_ms": round(prof, 4), "fwd_ms": round(fwdf, 4), "fwd_ms_median": round(fwdf_med, 4),
+            "fwd_ms_min": round(fwdf_min, 4), "gpu_launches_per_step": 2,
+            "path": "jattn_rope_qkv (fp16) + jattn_fwd_bf16: fp16 operands, no range scales, no Q.K^T correction "
+                    "(max-abs above 2e-2 on the outlier workloads)",
+            "roofline": tensor_roofline(flops, fwdf, peaks, peak_src, False, FWD_TRAFFIC_BYTES if full else None,
+                                        "attn_fwd_kernel<128, fp16 operands>")}
     fp8 = None
     if not args.no_fp8:
         ms8, pro8, fwd8, fwd8_med, fwd8_min = measure_path(jattn, ctx, w, dinp, "fp8", args.steps, args.warmup)
@@ -320,21 +327,26 @@ def run_ours(args, rank, world, local):
         "scaling": "strong", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
         "config": {"workload": w.name, "B": B, "H": H, "S": S, "S_txt": w.S_txt, "S_img": w.S_img,
                    "S_ref": w.S_ref, "d": d, "rope_split": list(w.split), "theta": w.theta,
-                   "path": "bf16 in/out, fp16 MMA operands, fp32 accumulate (jattn_rope_qkv + jattn_fwd_bf16)",
+                   "path": "bf16 in/out; jattn_rope_qkv_hp + jattn_fwd_bf16_hp: fp16 MMA operands with "
+                           "power-of-two block range scales and split-precision Q.K^T on 4 channel pairs per head, "
+                           "fp32 accumulate",
                    "l2": "inputs larger than L2 (623 MB qkv streams, 622 MB laid-out q/k/v)",
                    "parallelism": "single GPU"},
         "prologue_ms": round(pro_ms, 4), "fwd_ms": round(fwd_ms, 4), "fwd_ms_median": round(fwd_med, 4),
         "fwd_ms_min": round(fwd_min, 4),
-        "roofline": tensor_roofline(flops, fwd_ms, peaks, peak_src, False, FWD_TRAFFIC_BYTES if full else None,
-                                    "attn_fwd_kernel<128, fp16 operands>"),
-        "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / pro_ms / 1e6, 1),
+        "roofline": tensor_roofline(flops, fwd_ms, peaks, peak_src, False, None,
+                                    "attn_fwd_kernel<128, fp16 operands, high precision>"),
+        "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / prof / 1e6, 1),
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                              "frac": round(prologue_bytes(w, 2) / pro_ms / 1e6 / peaks["hbm_gbs"], 4),
-                              "peak_note": f"{peak_src} HBM copy bandwidth"},
-        "gpu_launches": 2 * args.steps,
+                              "frac": round(prologue_bytes(w, 2) / prof / 1e6 / peaks["hbm_gbs"], 4),
+                              "peak_note": f"{peak_src} HBM copy bandwidth",
+                              "kernel": "rope_qkv_kernel<128, fp16 out> (the fast path's prologue, one launch); "
+                                        "the headline's prologue stage (prologue with range scales and pair "
+                                        "statistics, pair selection, correction rows) is prologue_ms"},
+        "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
-    line["bf16_hp"] = hp
+    line["bf16_fast"] = fast
     if fp8 is not None:
         line["fp8"] = fp8
     line.update(extras)
@@ -497,7 +509,7 @@ def run_partition(args, rank, world, local):
     pos = inp["pos"].to(dev)
 
     def step(ev):
-        ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g])
+        ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g], precise=True)
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -511,11 +523,11 @@ def run_partition(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
         "scaling": "strong", "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "H": w.H, "S": w.S, "d": w.d,
-                   "path": "bf16 in/out, fp16 MMA operands; ulysses_attention (NCCL all-to-all, rope, forward, "
-                           "all-to-all) per rank",
+                   "path": "bf16 in/out; ulysses_attention per rank: NCCL all-to-all, jattn_rope_qkv_hp + "
+                           "jattn_fwd_bf16_hp, all-to-all",
                    "l2": "inputs larger than L2",
                    "parallelism": f"cfg{cfg} x ulysses{uly}"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clocks,
     }
     if rank == 0:

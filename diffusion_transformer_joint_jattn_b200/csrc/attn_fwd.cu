@@ -360,6 +360,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     bool ok = true;
 
     float sq = 1.f, max_sv = 1.f;
+    bool unit_scales = false;
     const float* sc_k = nullptr;
     const float* sc_v = nullptr;
     if constexpr (SCALED) {
@@ -370,10 +371,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       sc_k = p.scales + plane + bhn;
       sc_v = p.scales + 2 * plane + bhn;
       float mv = 0.f;
-      for (int j = lane; j < p.n_kv; j += 32) mv = fmaxf(mv, sc_v[j]);   // every tile: ratios stay <= 1
+      bool unit = sq == 1.f;
+      for (int j = lane; j < p.n_kv; j += 32) {         // every tile: ratios stay <= 1
+        const float a = sc_v[j];
+        mv = fmaxf(mv, a);
+        if constexpr (HP) unit = unit && a == 1.f && sc_k[j] == 1.f;
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
       max_sv = mv > 0.f ? mv : 1.f;
+      // HP with every range scale 1 (all ordinary inputs): the tiles need no
+      // per-tile scale (uniform across the warp).
+      if constexpr (HP) unit_scales = __all_sync(0xffffffffu, unit);
     }
     // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
     // exceeds the e4m3 range while p <= 2^8.  HP: as p * (s_v,j / max s_v)
@@ -393,7 +402,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const int kt = kt_cur;
       if (j + 1 < n_kv) kt_cur = kv_tile(j + 1);
       float c_j = sl2, bias = 0.f;
-      if constexpr (SCALED) {
+      if (SCALED && !unit_scales) {
         c_j = sl2 * sq * sk_nxt;
         bias = __log2f(sv_nxt / max_sv) + p8_log2;
         if (j + 1 < n_kv) {

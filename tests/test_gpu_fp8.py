@@ -1,18 +1,26 @@
-"""GPU parity of the FP8 path (jattn_rope_qkv e4m3 + jattn_fwd_fp8).
+"""GPU parity of the FP8 path (jattn_rope_qkv e4m3 + jattn_fwd_fp8) and of
+the FP8 path with token repair at full size.
 
 What is checked, and against what:
   * The quantised operands are checked bit-for-bit in test_gpu_rope.py.
   * The forward kernel is checked against the FP64 oracle run on the SAME
     dequantised operands with an exact softmax ("dequantised-operand
     oracle").  What separates the two is only the kernel's rounding of the
-    probabilities P to e4m3 (relative step 2^-4 in the normal range) and fp32
-    accumulation, so rel-L2 <= 5e-2 there (the measured level is about 2.5e-2;
-    an error in the scale handling shows up at 1e-1 and above).
+    probabilities P to e4m3 (3 mantissa bits, relative step 2^-4) and fp32
+    accumulation: measured 2.5e-2 .. 2.8e-2 on every case, bar 3e-2.  (An
+    emulation of the P rounding alone, with exact logits, gives 2.1e-2 ..
+    2.7e-2 whatever headroom P keeps below 448, so the bar cannot go lower
+    for e4m3 P.)
   * Closed-form cases (Q = 0, chosen per-block V scales): the output is the
     scale-weighted mean of V, exact up to the bf16 output rounding.
   * Against the exact FP64 result on the original bf16 inputs the error is
-    the e4m3 format floor of Q/K/V; it is measured and reported, with a loose
-    sanity bound (see the design notes for the per-workload floors).
+    the e4m3 format floor of Q/K/V, far above the 3e-2 target for plain FP8;
+    each workload is held to 1.1 x its measured floor.
+  * The FP8 path with the pages' token repair meets the 3e-2 target where
+    the repair budget rho reaches it (i2i_2048_base at rho = 0.005,
+    t2i_2048_base at 0.01, t2i_2048_distilled at 0.05) and is held to 1.1 x
+    its measured error where it does not (rho = 0.005 on the two t2i
+    workloads).
 """
 import math
 
@@ -23,11 +31,16 @@ import torch
 import oracle
 from diffusion_transformer_joint_jattn_b200 import jattn
 from diffusion_transformer_joint_jattn_b200 import workloads as W
-from parity_util import gather_lse, gather_rows, rel_l2, to_device, workload_case
+from parity_util import FP8_REL_L2, gather_lse, gather_rows, rel_l2, to_device, workload_case
 
 pytestmark = pytest.mark.gpu
 
-KERNEL_VS_DEQUANT = 5e-2
+KERNEL_VS_DEQUANT = 3e-2
+# Plain FP8 against the exact result: the e4m3 floor of Q/K/V.  No-outlier
+# d = 64 / 128 cases measure 5.3e-2 .. 5.6e-2; the workloads' floors below.
+SMALL_VS_EXACT = 6.2e-2
+WORKLOAD_VS_EXACT = {"t2i_2048_base": 1.1 * 9.48e-2, "t2i_2048_distilled": 1.1 * 2.83e-1,
+                     "i2i_2048_base": 1.1 * 8.78e-2}
 
 
 def _run(w, inp, dev):
@@ -66,7 +79,7 @@ def test_fp8_kernel_against_dequantised_operands(cuda_device, case):
     O, _ = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
     r = rel_l2(got, O)
     print(f"{case}: rel-L2 vs dequantised-operand oracle {r2:.3e}, vs exact {r:.3e}")
-    assert r <= 0.15
+    assert r <= SMALL_VS_EXACT
     assert jattn.device_status()[0] == jattn.OK
 
 
@@ -84,10 +97,11 @@ def test_fp8_with_qk_norm(cuda_device):
     dq, dk, dv = (_dequant(t, sc[i]) for i, t in enumerate((q8, k8, v8)))
     O2, _ = oracle.attention_on(dq, dk, dv)
     got = gather_rows(o, torch.arange(w.S).expand(w.B, w.H, w.S))
-    assert rel_l2(got, O2) <= KERNEL_VS_DEQUANT
     O, _ = oracle.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
                                   norm_w=nw, eps=1e-6)
-    assert rel_l2(got, O) <= 0.15
+    print(f"fp8 with query/key norm: vs dequantised-operand oracle {rel_l2(got, O2):.3e}, vs exact {rel_l2(got, O):.3e}")
+    assert rel_l2(got, O2) <= KERNEL_VS_DEQUANT
+    assert rel_l2(got, O) <= SMALL_VS_EXACT
 
 
 @pytest.mark.parametrize("sv", [(1.0, 1.0), (1.0, 0.5), (0.5, 1.0), (1.0, 0.25), (2.0 ** -6, 1.0), (1.0, 0.125),
@@ -134,5 +148,43 @@ def test_workload_fp8_sampled_rows(cuda_device, name):
     r2, r = rel_l2(got, O2), rel_l2(got, O)
     print(f"{name}: rel-L2 vs dequantised-operand oracle {r2:.3e}, vs exact (format floor) {r:.3e}")
     assert r2 <= KERNEL_VS_DEQUANT
-    assert r <= 0.5
+    assert r <= WORKLOAD_VS_EXACT[name]
     assert jattn.device_status()[0] == jattn.OK
+
+
+# (workload, rho, bar against the exact result): FP8_REL_L2 where the repair
+# budget reaches it, else 1.1 x the measured error at that budget.
+REPAIR_CASES = [("t2i_2048_base", 0.005, 1.1 * 3.23e-2), ("t2i_2048_base", 0.01, FP8_REL_L2),
+                ("t2i_2048_distilled", 0.005, 1.1 * 1.83e-1), ("t2i_2048_distilled", 0.05, FP8_REL_L2),
+                ("i2i_2048_base", 0.005, FP8_REL_L2)]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("name,rho,bar", REPAIR_CASES, ids=lambda x: str(x))
+def test_workload_fp8_repair_against_exact(cuda_device, name, rho, bar):
+    """The FP8 path with token repair at full size in the bench's launch
+    configuration, against the exact FP64 attention on 8 heads x 512 sampled
+    rows (the oracle rotates each checked head's keys in FP64)."""
+    w = W.BY_NAME[name]
+    inp = W.make_inputs(w, 0)
+    d = to_device(inp, cuda_device)
+    o = jattn.fwd_fp8_repair(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, rho=rho)
+    torch.cuda.synchronize()
+    assert jattn.device_status()[0] == jattn.OK
+    o = o.cpu()
+    qkv = torch.cat([t for t in (inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"]) if t is not None], dim=1)
+    pos = inp["pos"].numpy()
+    rows = W.sample_rows(w, 512, 3)
+    num = den = 0.0
+    for bh in range(0, w.B * w.H, max(1, w.B * w.H // 8)):
+        b, h = divmod(bh, w.H)
+        x = qkv[b, :, :, h].to(torch.float64).numpy()
+        k = oracle.rope_rotate(x[:, 1], pos, w.split, w.theta)
+        rr = rows[b, h].numpy()
+        q = oracle.rope_rotate(x[rr, 0], pos[rr], w.split, w.theta)
+        O, _ = oracle.attention_rows(q, k, x[:, 2], 1 / math.sqrt(w.d))
+        num += np.sum((o[b, rr, h].double().numpy() - O) ** 2)
+        den += np.sum(O ** 2)
+    r = math.sqrt(num / den)
+    print(f"{name} rho {rho}: FP8 with repair vs exact {r:.4e} (bar {bar:.3e})")
+    assert r <= bar

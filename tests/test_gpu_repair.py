@@ -5,7 +5,7 @@
   vs fp64 sums may reorder near-equal scores at the boundary, so the check is
   "every selected score >= every unselected score" within 1e-5 relative).
 * Output: against the oracle's repaired attention on the SAME set, with the
-  oracle's own e4m3 quantisation of Q/K/V: rel-L2 <= 5e-2 (what separates
+  oracle's own e4m3 quantisation of Q/K/V: rel-L2 <= 3e-2 (what separates
   them is the kernel's e4m3 rounding of P, as for the plain FP8 path); LSE
   within 2e-3.
 * rho = 0 reproduces the plain FP8 path bit for bit; rho = 1 repairs every
@@ -78,7 +78,7 @@ def test_repair_selection_and_parity(cuda_device, case, rho):
     got = gather_rows(o, rows)
     r = rel_l2(got, O)
     print(f"{case} rho={rho} n={n}: rel-L2 vs repaired oracle {r:.3e}")
-    assert r <= 5e-2
+    assert r <= 3e-2
     np.testing.assert_allclose(gather_lse(lse, rows), L, rtol=0, atol=2e-3)
     assert jattn.device_status()[0] == jattn.OK
 
@@ -122,7 +122,7 @@ def test_repair_with_qk_norm(cuda_device):
     _check_selection(rep, oracle.repair_scores(k, v), oracle.repair_count(w.S, 0.05))
     O, _ = oracle.repaired_attention(q, k, v, _deq(q), _deq(k), _deq(v), rep)
     got = gather_rows(o, torch.arange(w.S).expand(w.B, w.H, w.S))
-    assert rel_l2(got, O) <= 5e-2
+    assert rel_l2(got, O) <= 3e-2
 
 
 @pytest.mark.parametrize("name", ["t2i_1024_base", "t2i_2048_distilled"])
@@ -150,7 +150,7 @@ def test_repair_full_size_2048(cuda_device):
     """t2i_2048_base at full size in the bench's launch configuration
     (B = 2, H = 24, S = 16896, rho = 0.005 -> 85 tokens per head); 8 of the
     48 heads are checked against the oracle on 512 sampled rows each: valid
-    top-n selection, rel-L2 <= 5e-2 against the repaired-attention oracle,
+    top-n selection, rel-L2 <= 3e-2 against the repaired-attention oracle,
     and closer to the exact result than the plain FP8 path."""
     w = W.BY_NAME["t2i_2048_base"]
     inp = W.make_inputs(w, 0)
@@ -196,5 +196,5 @@ def test_repair_full_size_2048(cuda_device):
     r_rep, r_plain = np.sqrt(num_exact_rep / den), np.sqrt(num_plain / den)
     print(f"t2i_2048_base repair: vs repaired oracle {r_vs_oracle:.3e}; vs exact: repaired {r_rep:.3e}, "
           f"plain FP8 {r_plain:.3e}")
-    assert r_vs_oracle <= 5e-2
+    assert r_vs_oracle <= 3e-2
     assert r_rep < r_plain
