@@ -43,6 +43,9 @@ WORKLOAD = "t2i_2048_base"
 # and O once each, linear in tokens).
 FWD_TRAFFIC_BYTES = 205.21e6 * 16896 / 4608
 FWD_FP8_TRAFFIC_BYTES = 109.19e6 * 16896 / 4608
+# The high-precision instance (the headline's forward): 184.13 MB read +
+# 35.79 MB written on t2i_1024_base (profiles/attn_fwd_hp_t2i_1024_base.md).
+FWD_HP_TRAFFIC_BYTES = (184.13e6 + 35.79e6) * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 # Per-sample time of the oracle on the host cores (both CPU legs use the same
@@ -334,7 +337,7 @@ def run_ours(args, rank, world, local):
                    "parallelism": "single GPU"},
         "prologue_ms": round(pro_ms, 4), "fwd_ms": round(fwd_ms, 4), "fwd_ms_median": round(fwd_med, 4),
         "fwd_ms_min": round(fwd_min, 4),
-        "roofline": tensor_roofline(flops, fwd_ms, peaks, peak_src, False, None,
+        "roofline": tensor_roofline(flops, fwd_ms, peaks, peak_src, False, FWD_HP_TRAFFIC_BYTES if full else None,
                                     "attn_fwd_kernel<128, fp16 operands, high precision>"),
         "prologue_roofline": {"bound": "hbm", "achieved": round(prologue_bytes(w, 2) / prof / 1e6, 1),
                               "peak": peaks["hbm_gbs"], "unit": "GB/s",

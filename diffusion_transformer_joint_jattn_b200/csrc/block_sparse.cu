@@ -15,10 +15,11 @@
 // Two launches:
 //   block_pool_kernel    column sums of every 128-token tile of Q and K
 //                        (coalesced 16-byte loads, one CTA per tile);
-//   block_select_kernel  one CTA per (b, h, query block): the shares, the
-//                        threshold, and the kept key tiles compacted in
-//                        ascending order -> kv_list / kv_count, which the
-//                        forward kernel walks instead of every key tile.
+//   block_select_kernel  one CTA per (b, h, query block): the block logits
+//                        (a warp per key block), the shares, the threshold,
+//                        and the kept key tiles compacted in ascending order
+//                        -> kv_list / kv_count, which the forward kernel
+//                        walks instead of every key tile.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_fp16.h>
@@ -91,68 +92,74 @@ __device__ __forceinline__ float block_reduce(float v, float* red, bool is_max) 
 }
 
 // grid (n_qb, B*H): one query block of 256 tokens (two 128-token tiles).
+// The block logits are computed a warp per key block (coalesced float4 reads
+// of the key block's column sums, a shuffle reduction) into this CTA's row
+// of p.logits, then read back coalesced for the max, the softmax
+// denominator and the threshold.
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SparseParams p) {
-  __shared__ float qbar[D];
-  __shared__ float red[kSelThreads / 32];
-  __shared__ int wcount[kSelThreads / 32];
+  constexpr int NW = kSelThreads / 32;
+  constexpr int CPL = D / 32;                  // channels per lane (4 or 2)
+  __shared__ __align__(16) float qbar[D];
+  __shared__ float red[NW];
+  __shared__ float wmx[NW];
+  __shared__ int warg[NW];
+  __shared__ int wcount[NW];
   const int I = blockIdx.x, bh = blockIdx.y, tid = threadIdx.x;
   const int lane = tid & 31, warp = tid >> 5;
   const int n_qb = gridDim.x, n_kb = p.nblk;
   const int r_lo = I * 2 * JATTN_BLOCK, r_hi = min(p.S, r_lo + 2 * JATTN_BLOCK);
   const float* pq = p.pool + (static_cast<size_t>(bh) * p.nblk) * D;
   const float* pk = p.pool + (static_cast<size_t>(p.BH) + bh) * p.nblk * D;
+  float* lg = p.logits + (static_cast<size_t>(bh) * n_qb + I) * n_kb;
   if (tid < D) {
     float s = pq[static_cast<size_t>(2 * I) * D + tid];
     if (2 * I + 1 < p.nblk) s += pq[static_cast<size_t>(2 * I + 1) * D + tid];
     qbar[tid] = s / static_cast<float>(r_hi - r_lo);
   }
   __syncthreads();
-  // Logit of key block J: qbar . kbar_J * scale (recomputed in each pass;
-  // n_kb * D multiply-adds per pass).
-  auto logit = [&](int J) {
-    const float* kr = pk + static_cast<size_t>(J) * D;
-    float s = 0.f;
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) s = fmaf(qbar[c], kr[c], s);
-    const int n = min(p.S - J * JATTN_BLOCK, JATTN_BLOCK);
-    return s / static_cast<float>(n) * p.scale;
-  };
-  // pass 1: the largest logit and its (lowest) block
+  // logits qbar . kbar_J * scale; the largest and its (lowest) block
   float mx = -INFINITY;
   int arg = 0x7fffffff;
-  for (int J = tid; J < n_kb; J += kSelThreads) {
-    const float s = logit(J);
-    if (s > mx) { mx = s; arg = J; }
-  }
+  for (int J = warp; J < n_kb; J += NW) {
+    const float* kr = pk + static_cast<size_t>(J) * D + lane * CPL;
+    float s = 0.f;
+    if constexpr (CPL == 4) {
+      const float4 k4 = *reinterpret_cast<const float4*>(kr);
+      const float4 q4 = *reinterpret_cast<const float4*>(qbar + lane * CPL);
+      s = fmaf(q4.x, k4.x, fmaf(q4.y, k4.y, fmaf(q4.z, k4.z, q4.w * k4.w)));
+    } else {
+      const float2 k2 = *reinterpret_cast<const float2*>(kr);
+      const float2 q2 = *reinterpret_cast<const float2*>(qbar + lane * CPL);
+      s = fmaf(q2.x, k2.x, q2.y * k2.y);
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    const float om = __shfl_xor_sync(0xffffffffu, mx, o);
-    const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-    if (om > mx || (om == mx && oa < arg)) { mx = om; arg = oa; }
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    const int n = min(p.S - J * JATTN_BLOCK, JATTN_BLOCK);
+    s = s / static_cast<float>(n) * p.scale;
+    if (lane == 0) lg[J] = s;
+    if (s > mx) { mx = s; arg = J; }               // warp-uniform: every lane holds s
   }
-  __shared__ float wmx[kSelThreads / 32];
-  __shared__ int warg[kSelThreads / 32];
   if (lane == 0) { wmx[warp] = mx; warg[warp] = arg; }
-  __syncthreads();
+  __syncthreads();                                  // also orders the logit writes before the reads below
   mx = wmx[0];
   arg = warg[0];
 #pragma unroll
-  for (int w = 1; w < kSelThreads / 32; ++w)
+  for (int w = 1; w < NW; ++w)
     if (wmx[w] > mx || (wmx[w] == mx && warg[w] < arg)) { mx = wmx[w]; arg = warg[w]; }
-  // pass 2: the softmax denominator
+  // the softmax denominator
   float den = 0.f;
-  for (int J = tid; J < n_kb; J += kSelThreads) den += expf(logit(J) - mx);
+  for (int J = tid; J < n_kb; J += kSelThreads) den += expf(lg[J] - mx);
   den = block_reduce(den, red, false);
-  // pass 3: keep share >= tau / n_kb, i.e. exp(s - mx) >= den * tau / n_kb,
-  // and the largest; write the kept blocks in ascending order.
+  // keep share >= tau / n_kb, i.e. exp(s - mx) >= den * tau / n_kb, and the
+  // largest; write the kept blocks in ascending order.
   const float cut = den * p.tau / static_cast<float>(n_kb);
   int32_t* list = p.kv_list + (static_cast<size_t>(bh) * n_qb + I) * n_kb;
   int base = 0;
   for (int J0 = 0; J0 < n_kb; J0 += kSelThreads) {
     const int J = J0 + tid;
     bool keep = false;
-    if (J < n_kb) keep = J == arg || expf(logit(J) - mx) >= cut;
+    if (J < n_kb) keep = J == arg || expf(lg[J] - mx) >= cut;
     const uint32_t bal = __ballot_sync(0xffffffffu, keep);
     if (lane == 0) wcount[warp] = __popc(bal);
     __syncthreads();
@@ -161,7 +168,7 @@ __global__ void __launch_bounds__(kSelThreads) block_select_kernel(const SparseP
     if (keep) list[off + __popc(bal & ((1u << lane) - 1u))] = J;
     int tot = 0;
 #pragma unroll
-    for (int w = 0; w < kSelThreads / 32; ++w) tot += wcount[w];
+    for (int w = 0; w < NW; ++w) tot += wcount[w];
     base += tot;
     __syncthreads();
   }

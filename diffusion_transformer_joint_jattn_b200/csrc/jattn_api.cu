@@ -434,7 +434,7 @@ jattn_status jattn_fwd_bf16_hp(const jattn_shape* shape, const void* q, const vo
 namespace {
 
 struct SparseLayout {
-  size_t pool, list, count, total;
+  size_t pool, logits, list, count, total;
 };
 
 SparseLayout sparse_layout(const jattn_shape* shape) {
@@ -445,6 +445,7 @@ SparseLayout sparse_layout(const jattn_shape* shape) {
   size_t off = 0;
   auto seg = [&](size_t bytes) { const size_t at = off; off += align256(bytes); return at; };
   L.pool = seg(2 * BH * nb * d * 4);
+  L.logits = seg(BH * nq * nb * 4);
   L.list = seg(BH * nq * nb * 4);
   L.count = seg(BH * nq * 4);
   L.total = off;
@@ -487,6 +488,7 @@ jattn_status jattn_fwd_block_sparse(const jattn_shape* shape, jattn_dtype in_dty
   sp.scale = p.scale_log2 / 1.4426950408889634f;
   sp.tau = tau;
   sp.pool = reinterpret_cast<float*>(ws + L.pool);
+  sp.logits = reinterpret_cast<float*>(ws + L.logits);
   sp.kv_list = kv_list != nullptr ? kv_list : reinterpret_cast<int32_t*>(ws + L.list);
   sp.kv_count = kv_count != nullptr ? kv_count : reinterpret_cast<int32_t*>(ws + L.count);
   if (jattn::launch_block_select(sp, in_dtype == JATTN_BF16, cs) != cudaSuccess) return JATTN_ERR_CUDA;

@@ -88,6 +88,7 @@ struct SparseParams {
   float scale;                  // softmax scale
   float tau;                    // keep a key block iff its estimated share >= tau / nblk
   float* pool;                  // [2][B*H][nblk][d] column sums of every 128-token tile of Q, K
+  float* logits;                // [B*H][n_qb][nblk] block logits (scratch of the selection)
   int32_t* kv_list;             // [B*H][n_qb][nblk] kept key tiles, ascending (first kv_count entries)
   int32_t* kv_count;            // [B*H][n_qb]
 };
