@@ -149,6 +149,7 @@ jattn_status rope_common(const jattn_shape* shape, const void* qkv_txt, const vo
   p.nblk = n_blocks(p.S);
   p.pos = pos;
   p.theta = static_cast<double>(theta);
+  p.rope = jattn::make_rope_table(p.theta, p.split, p.d);
   p.dst[0] = q;
   p.dst[1] = k;
   p.dst[2] = v;
@@ -395,6 +396,7 @@ jattn_status jattn_rope_qkv_hp(const jattn_shape* shape, const void* qkv_txt, co
   c.nblk = n_blocks(c.S);
   c.pos = pos;
   c.theta = static_cast<double>(theta);
+  c.rope = jattn::make_rope_table(c.theta, c.split, c.d);
   c.norm_w = norm_w;
   c.norm_r = norm_w != nullptr ? norm_r : nullptr;
   c.scales = scales;
@@ -563,6 +565,7 @@ jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt,
     g.n = n;
     g.pos = pos;
     g.theta = static_cast<double>(theta);
+    g.rope = jattn::make_rope_table(g.theta, g.split, g.d);
     g.norm_w = norm_w;
     g.eps = eps;
     g.idx = idx;

@@ -2,12 +2,36 @@
 // and the kernel translation units.  Not part of the public interface.
 #pragma once
 
+#include <cmath>
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
 namespace jattn {
+
+// Rotary frequencies of the d/2 channel pairs, built on the host once per
+// call: pair p lies on axis axis[p] (0 = t, 1 = row, 2 = col: spans of
+// split[0], split[1], split[2] channels in that order) and turns by
+// pos_axis * omega[p], omega[p] = theta^(-2i/n) for its index i inside its
+// axis span of n channels.  Passed by value in the kernel parameters.
+struct RopeTable {
+  double omega[64];
+  uint8_t axis[64];
+};
+
+inline RopeTable make_rope_table(double theta, const int split[3], int d) {
+  RopeTable t{};
+  for (int p = 0; p < d / 2 && p < 64; ++p) {
+    int axis, i, n;
+    if (p < split[0] / 2) { axis = 0; i = p; n = split[0]; }
+    else if (p < (split[0] + split[1]) / 2) { axis = 1; i = p - split[0] / 2; n = split[1]; }
+    else { axis = 2; i = p - (split[0] + split[1]) / 2; n = split[2]; }
+    t.axis[p] = static_cast<uint8_t>(axis);
+    t.omega[p] = std::pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(n));
+  }
+  return t;
+}
 
 struct RopeParams {
   const __nv_bfloat16* src[3];  // txt, img, ref streams [B, S_part, 3, H, d]
@@ -16,6 +40,7 @@ struct RopeParams {
   const int32_t* pos;           // [S, 3]
   double theta;
   int split[3];
+  RopeTable rope;               // frequencies of theta / split (make_rope_table)
   void* dst[3];                 // q, k, v [B, H, S, d]
   float* scales;                // e4m3 output: [3][B][H][nblk]
   const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
@@ -37,6 +62,7 @@ struct GatherParams {
   const int32_t* pos;           // [S, 3]
   double theta;
   int split[3];
+  RopeTable rope;
   const float* norm_w;          // as RopeParams
   float eps;
   const int32_t* idx;           // [B*H][n] token indices
@@ -68,6 +94,7 @@ struct CorrParams {
   const int32_t* pos;           // [S, 3]
   double theta;
   int split[3];
+  RopeTable rope;
   const float* norm_w;          // query/key RMSNorm weights [3][2][d], or null
   const float* norm_r;          // with norm_w: [2][B*H][S] row factors written by the prologue
   const float* scales;          // [3][B][H][nblk] power-of-two range scales written by the prologue

@@ -128,11 +128,8 @@ __global__ void __launch_bounds__(JATTN_BLOCK) qk_correct_kernel(const CorrParam
   for (int k = 0; k < kCorrPairs; ++k) pairs[k] = p.sel[static_cast<size_t>(bh) * kCorrPairs + k];
   float cs[kCorrPairs], sn[kCorrPairs];
 #pragma unroll
-  for (int k = 0; k < kCorrPairs; ++k) {
-    int axis, ii, n;
-    pair_axis(pairs[k], p.split[0], p.split[1], p.split[2], axis, ii, n);
-    pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs[k], sn[k]);
-  }
+  for (int k = 0; k < kCorrPairs; ++k)
+    angle_cos_sin(p.pos[3 * t + p.rope.axis[pairs[k]]], p.rope.omega[pairs[k]], cs[k], sn[k]);
   const size_t BHS = static_cast<size_t>(p.BH) * p.S;
 #pragma unroll
   for (int which = 0; which < 2; ++which) {

@@ -27,22 +27,16 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&x)[8]) {
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t u) { return __uint_as_float(static_cast<uint32_t>(u) << 16); }
 
-// Axis, index inside the axis span and span width of channel pair `pair`
-// (0 .. d/2-1); spans are laid out t, row, col.
-__device__ __forceinline__ void pair_axis(int pair, int n0, int n1, int n2, int& axis, int& i, int& n) {
-  if (pair < n0 / 2) { axis = 0; i = pair; n = n0; }
-  else if (pair < (n0 + n1) / 2) { axis = 1; i = pair - n0 / 2; n = n1; }
-  else { axis = 2; i = pair - (n0 + n1) / 2; n = n2; }
-}
-
-// cos/sin of pos_axis * theta^(-2i/n): the angle is formed and reduced to
-// [-pi, pi] in fp64, then rotated with the fp32 sincos.
-__device__ __forceinline__ void pair_cos_sin(int32_t pos_axis, int i, int n, double theta,
-                                             float& c, float& s) {
-  const double omega = pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(n));
+// cos/sin of the angle pos_axis * omega of one channel pair: the angle is
+// formed and reduced to [-pi, pi] in fp64 (multiplying by 1/(2 pi)), then
+// rotated with the fp32 sincos.  omega comes from the RopeTable the host
+// builds once per call (see jattn_internal.h), so every kernel that rotates
+// the same pair of the same token gets the same cos/sin bits.
+__device__ __forceinline__ void angle_cos_sin(int32_t pos_axis, double omega, float& c, float& s) {
   const double ang = static_cast<double>(pos_axis) * omega;
   const double two_pi = 6.283185307179586476925286766559;
-  const double r = ang - rint(ang / two_pi) * two_pi;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  const double r = ang - rint(ang * inv_two_pi) * two_pi;
   sincosf(static_cast<float>(r), &s, &c);
 }
 

@@ -93,7 +93,6 @@ rope_qkv_kernel(const RopeParams p) {
   const int blk = blockIdx.x;
   const int b = blockIdx.y;
   const int H = p.H, S = p.S;
-  const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
   if constexpr (NORM) {
     for (int i = tid; i < 6 * D; i += NT) wsm[i] = p.norm_w[i];
     __syncthreads();
@@ -124,9 +123,8 @@ rope_qkv_kernel(const RopeParams p) {
       cs[i][j] = 1.f;
       sn[i][j] = 0.f;
       if (valid[i]) {
-        int axis, ii, n;
-        pair_axis(cg * 4 + j, n0, n1, n2, axis, ii, n);
-        pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs[i][j], sn[i][j]);
+        const int pair = cg * 4 + j;
+        angle_cos_sin(p.pos[3 * t + p.rope.axis[pair]], p.rope.omega[pair], cs[i][j], sn[i][j]);
       }
     }
   }
@@ -434,13 +432,11 @@ __global__ void __launch_bounds__(256) repair_gather_kernel(const GatherParams p
 #pragma unroll
     for (int e = 0; e < CPL; ++e) k[e] = norm_scale(k[e], rr, w[e]);
   }
-  const int n0 = p.split[0], n1 = p.split[1], n2 = p.split[2];
 #pragma unroll
   for (int j = 0; j < CPL / 2; ++j) {
-    int axis, ii, n;
-    pair_axis(c0 / 2 + j, n0, n1, n2, axis, ii, n);
+    const int pair = c0 / 2 + j;
     float cs, sn;
-    pair_cos_sin(p.pos[3 * t + axis], ii, n, p.theta, cs, sn);
+    angle_cos_sin(p.pos[3 * t + p.rope.axis[pair]], p.rope.omega[pair], cs, sn);
     rotate_pair(k[2 * j], k[2 * j + 1], cs, sn, k[2 * j], k[2 * j + 1]);
   }
   bool range_hit = false;
