@@ -153,7 +153,9 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 // HP (KIND 0 only): the high-precision 16-bit path -- per-block power-of-two
 // range scales of Q, K and V folded in like the e4m3 block scales, and each
 // logit tile completed by Qc . Kc^T over the correction tiles (tmQc, tmKc).
-template <int D, int KIND, bool HP>
+// SPARSE: walk the CTA's key-tile list (block-sparse attention) instead of
+// every key tile; a separate instance so the dense ones carry no list state.
+template <int D, int KIND, bool HP, bool SPARSE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQc,
@@ -181,11 +183,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const int b = bh / p.H, h = bh % p.H;
   // Key tiles this CTA walks: all n_kv in order, or (block-sparse) the
   // first kv_count entries of its kv_list row.
-  const int32_t* kv_list = p.kv_list != nullptr
-                               ? p.kv_list + (static_cast<size_t>(bh) * gridDim.x + qp) * p.n_kv
-                               : nullptr;
-  const int n_kv = kv_list != nullptr ? p.kv_count[static_cast<size_t>(bh) * gridDim.x + qp] : p.n_kv;
-  auto kv_tile = [&](int j) { return kv_list != nullptr ? __ldg(kv_list + j) : j; };
+  const int32_t* kv_list = SPARSE ? p.kv_list + (static_cast<size_t>(bh) * gridDim.x + qp) * p.n_kv : nullptr;
+  const int n_kv = SPARSE ? p.kv_count[static_cast<size_t>(bh) * gridDim.x + qp] : p.n_kv;
+  auto kv_tile = [&](int j) {
+    if constexpr (SPARSE) return __ldg(kv_list + j);
+    else return j;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(&bar->q_full, 1);
@@ -605,12 +608,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
-template <int D, int KIND, bool HP = false>
+template <int D, int KIND, bool HP = false, bool SPARSE = false>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tqc, const CUtensorMap& tkc, cudaStream_t st) {
   using C = Cfg<D, KIND == 2, HP>;
   static_assert(C::SMEM <= 232448, "shared memory budget");
-  auto kern = attn_fwd_kernel<D, KIND, HP>;
+  auto kern = attn_fwd_kernel<D, KIND, HP, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
   dim3 grid((p.n_tiles + NQ - 1) / NQ, p.B * p.H);
@@ -639,6 +642,13 @@ int fwd_kv_rows() { return BN; }
 
 cudaError_t launch_fwd_f16(const FwdParams& p, int d, bool in_bf16, const CUtensorMap& tq,
                            const CUtensorMap& tk, const CUtensorMap& tv, cudaStream_t st) {
+  if (p.kv_list != nullptr) {
+    if (in_bf16)
+      return d == 128 ? launch_t<128, 1, false, true>(p, tq, tk, tv, tq, tk, st)
+                      : launch_t<64, 1, false, true>(p, tq, tk, tv, tq, tk, st);
+    return d == 128 ? launch_t<128, 0, false, true>(p, tq, tk, tv, tq, tk, st)
+                    : launch_t<64, 0, false, true>(p, tq, tk, tv, tq, tk, st);
+  }
   if (in_bf16) return d == 128 ? launch_t<128, 1>(p, tq, tk, tv, tq, tk, st) : launch_t<64, 1>(p, tq, tk, tv, tq, tk, st);
   return d == 128 ? launch_t<128, 0>(p, tq, tk, tv, tq, tk, st) : launch_t<64, 0>(p, tq, tk, tv, tq, tk, st);
 }
