@@ -22,8 +22,10 @@
 //   warp 9      TMA producer: Q tiles once, K_j / V_j into smem rings.
 //   (warps 10, 11 idle: they complete the third warpgroup.)
 // The block starts at 168 registers per thread (384 x 168 = 64512); the
-// MMA/TMA warpgroup then releases registers down to 56 and the two softmax
-// warpgroups grow to 224 (2 x 128 x 224 + 128 x 56 = 64512).
+// MMA/TMA warpgroup then releases registers and the two softmax warpgroups
+// grow (224 / 56 for e4m3 operands, 216 / 72 for the high-precision
+// instance, 208 / 88 for the plain 16-bit one, 200 / 104 when walking a
+// key-tile list; 2 x 128 x softmax + 128 x other = 64512).
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256, 256+d), O_1 [384, 384+d).
 // Because the tensor pipe runs one thread's MMAs in order, the commit that
 // signals S_t(j) also proves PV_t(j-1) finished: O_t is stable for the
@@ -46,9 +48,19 @@ constexpr int BN = 128;              // keys per tile
 constexpr int kMmaWarp = 8;
 constexpr int kProducerWarp = 9;
 constexpr int kThreads = 384;
-constexpr uint32_t kRegsSoftmax = 224;
-constexpr uint32_t kRegsOther = 56;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsOther <= kThreads * 168, "register split");
+// Register split after setmaxnreg (multiples of 8, together exactly the
+// 384 x 168 the block launches with): ptxas allocates each role's code within
+// its share, and a spill in the single MMA-issuing thread sits on the
+// S -> P -> MMA chain, so each instance gets the split that leaves both its
+// softmax and its MMA / TMA code spill-free (checked with -Xptxas -v).
+template <int KIND, bool HP, bool SPARSE>
+__host__ __device__ constexpr uint32_t regs_softmax() {
+  return KIND == 2 ? 224u : (HP ? 216u : (SPARSE ? 200u : 208u));
+}
+template <int KIND, bool HP, bool SPARSE>
+__host__ __device__ constexpr uint32_t regs_other() {
+  return (kThreads * 168u - 2u * 128u * regs_softmax<KIND, HP, SPARSE>()) / 128u;
+}
 constexpr uint32_t kTmemCols = 512;
 // Lazy rescale: O and l are rescaled only when a row's running max grows by
 // more than this many log2 units, so P <= 2^threshold in between.  16-bit P
@@ -222,7 +234,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const WaitCtl ctl{&bar->abort, p.status, p.timeout_ns};
   if (warp >= 8) {
     // Third warpgroup: producer, MMA issuer and two idle warps.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsOther));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(regs_other<KIND, HP, SPARSE>()));
     if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -351,7 +363,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(regs_softmax<KIND, HP, SPARSE>()));
     const int t = warp >> 2;                          // query tile of this warpgroup
     const int row = (warp & 3) * 32 + lane;           // TMEM lane == row in the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
