@@ -483,8 +483,9 @@ def measure_e2e(jattn, ctx: Ctx, w, inp, steps, warmup, flops):
                        steps, warmup)
     return {"value": round(whole_job_tflops(flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 3),
             "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-            "api": "jattn.joint_attention -> jattn_joint_attention_host (C ABI, pinned host in/out, "
-                   "copies pipelined with the kernels in (batch entry, 2-head) chunks on copy streams)"}
+            "api": "jattn.joint_attention -> jattn_joint_attention_host (C ABI, pinned host in/out, the "
+                   "high-precision pair, copies pipelined with the kernels in (batch entry, 2-head) chunks on "
+                   "copy streams)"}
 
 
 # --------------------------------------------------------------------------- N > 1

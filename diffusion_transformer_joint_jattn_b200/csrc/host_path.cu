@@ -59,7 +59,7 @@ int head_groups(int H) {
 }
 
 struct HostLayout {
-  size_t part[3], pos, q, k, v, scales, o, total;
+  size_t part[3], pos, q, k, v, scales, scales_chunk, qc, kc, hp_ws, hp_ws_bytes, o, total;
 };
 
 bool valid_path(jattn_dtype path) { return path == JATTN_FP16 || path == JATTN_BF16 || path == JATTN_E4M3; }
@@ -80,7 +80,19 @@ HostLayout host_layout(const jattn_shape* s, jattn_dtype path) {
   L.q = seg(B * H * S * d * eb);
   L.k = seg(B * H * S * d * eb);
   L.v = seg(B * H * S * d * eb);
-  L.scales = seg(path == JATTN_E4M3 ? B * 3 * H * nb * 4 : 0);
+  // block scales (e4m3 scales, or the high-precision path's range scales),
+  // one 256-byte aligned slice per chunk
+  const size_t G = head_groups(s->H);
+  L.scales_chunk = path == JATTN_BF16 ? 0 : align256(3 * (H / G) * nb * 4);
+  L.scales = seg(B * G * L.scales_chunk);
+  // the high-precision path (JATTN_FP16): correction rows, and one scratch
+  // area of jattn_rope_qkv_hp that the chunks reuse in stream order
+  const bool hp = path == JATTN_FP16;
+  L.qc = seg(hp ? B * H * S * 16 * 2 : 0);
+  L.kc = seg(hp ? B * H * S * 16 * 2 : 0);
+  const jattn_shape one{1, static_cast<int>(H / G), s->S_txt, s->S_img, s->S_ref, s->d};
+  L.hp_ws_bytes = hp ? jattn_rope_qkv_hp_workspace(&one) : 0;
+  L.hp_ws = seg(L.hp_ws_bytes);
   L.o = seg(B * S * H * d * 2);
   L.total = off;
   return L;
@@ -135,7 +147,6 @@ extern "C" jattn_status jattn_joint_attention_host(const jattn_shape* shape, con
   const int G = head_groups(H), Hg = H / G;
   const int S = shape->S_txt + shape->S_img + shape->S_ref;
   const size_t eb = path == JATTN_E4M3 ? 1 : 2;
-  const size_t nb = (static_cast<size_t>(S) + JATTN_BLOCK - 1) / JATTN_BLOCK;
   const size_t row_in = static_cast<size_t>(H) * d * 2;          // host input: one (token, Q|K|V) row
   const size_t row_grp = static_cast<size_t>(Hg) * d * 2;        // the group's part of it
   const size_t lay_c = static_cast<size_t>(Hg) * S * d * eb;     // one chunk of laid-out q / k / v
@@ -168,9 +179,17 @@ extern "C" jattn_status jattn_joint_attention_host(const jattn_shape* shape, con
       const int32_t* dpos = reinterpret_cast<const int32_t*>(ws + L.pos);
       jattn_status st;
       if (path == JATTN_E4M3) {
-        float* sc = reinterpret_cast<float*>(ws + L.scales) + c * 3 * Hg * nb;
+        float* sc = reinterpret_cast<float*>(ws + L.scales + c * L.scales_chunk);
         st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], dpos, theta, split, JATTN_E4M3, q, k, v, sc, cs);
         if (st == JATTN_OK) st = jattn_fwd_fp8(&one, q, k, v, sc, oc, nullptr, softmax_scale, cs);
+      } else if (path == JATTN_FP16) {
+        // the high-precision 16-bit pair
+        float* sc = reinterpret_cast<float*>(ws + L.scales + c * L.scales_chunk);
+        void* qc = ws + L.qc + c * static_cast<size_t>(Hg) * S * 32;
+        void* kc = ws + L.kc + c * static_cast<size_t>(Hg) * S * 32;
+        st = jattn_rope_qkv_hp(&one, dparts[0], dparts[1], dparts[2], dpos, theta, split, nullptr, 0.f, q, k, v, sc,
+                               qc, kc, ws + L.hp_ws, L.hp_ws_bytes, cs);
+        if (st == JATTN_OK) st = jattn_fwd_bf16_hp(&one, q, k, v, sc, qc, kc, oc, nullptr, softmax_scale, cs);
       } else {
         st = jattn_rope_qkv(&one, dparts[0], dparts[1], dparts[2], dpos, theta, split, path, q, k, v, nullptr, cs);
         if (st == JATTN_OK) st = jattn_fwd_bf16(&one, path, q, k, v, oc, nullptr, softmax_scale, cs);

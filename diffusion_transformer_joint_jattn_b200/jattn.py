@@ -522,19 +522,22 @@ def fwd_fp8_repair_noalloc(qkv_txt, qkv_img, qkv_ref, pos, split: Sequence[int],
 
 
 def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.0, path: str = "bf16",
-                    operand_dtype: str = "fp16", want_lse: bool = False, out=None, stream=None,
-                    norm_w=None, eps: float = 1e-6, workspace=None, precise: bool = False):
-    """The whole hot path: rope_qkv -> fwd_bf16 (or rope_qkv e4m3 -> fwd_fp8),
-    with the query/key RMSNorm fused into rope_qkv when ``norm_w`` is given;
-    ``precise`` (device tensors, BF16 path) selects the high-precision pair
-    rope_qkv_hp -> fwd_bf16_hp.
+                    operand_dtype: str | None = None, want_lse: bool = False, out=None, stream=None,
+                    norm_w=None, eps: float = 1e-6, workspace=None, precise: bool = True):
+    """The whole hot path, with the query/key RMSNorm fused into the
+    prologue when ``norm_w`` is given.  path "bf16": the high-precision pair
+    rope_qkv_hp -> fwd_bf16_hp by default; ``precise=False`` selects the
+    plain pair rope_qkv -> fwd_bf16 with ``operand_dtype`` operands ("fp16"
+    unless given).  path "fp8": rope_qkv e4m3 -> fwd_fp8.
 
     CUDA tensors: the device entry points, asynchronous on ``stream``.
     CPU tensors (pinned for overlap): jattn_joint_attention_host, which
-    copies in, runs the path and copies O out pipelined over the batch; the
-    result lands in ``out`` (a bf16 [B, S, H, d] host tensor, allocated here
-    if None) and the call returns once it is there.  The host entry has no
-    LSE output and no norm; those need device tensors.
+    copies in, runs the path and copies O out pipelined over (batch entry,
+    head group) chunks; the result lands in ``out`` (a bf16 [B, S, H, d] host
+    tensor, allocated here if None) and the call returns once it is there.
+    Its plain 16-bit path takes bf16 operands (fp16 operands are those of the
+    high-precision pair).  The host entry has no LSE output and no norm;
+    those need device tensors.
     Returns O bf16 [B, S, H, d] (and LSE for device tensors)."""
     parts = [qkv_txt, qkv_img, qkv_ref]
     ref = next(t for t in parts if t is not None)
@@ -550,9 +553,16 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
         if pos.dtype != torch.int32 or not pos.is_contiguous():
             raise ValueError("pos must be a contiguous int32 tensor")
         S = sum(lens)
-        code = E4M3 if path == "fp8" else _NAME_CODE[operand_dtype]
         if path not in ("bf16", "fp8"):
             raise ValueError(f"unknown path {path!r}")
+        if path == "fp8":
+            code = E4M3
+        elif precise:
+            code = FP16                   # the host entry's high-precision pair
+        elif operand_dtype in (None, "bf16"):
+            code = BF16
+        else:
+            raise ValueError("the host entry's plain 16-bit path takes bf16 operands")
         shape = make_shape(B, H, lens[0], lens[1], lens[2], d)
         need = lib.jattn_joint_attention_host_workspace(ctypes.byref(shape), code)
         dev = torch.device("cuda", torch.cuda.current_device())
@@ -572,7 +582,8 @@ def joint_attention(qkv_txt, qkv_img, qkv_ref, pos, split, theta: float = 10000.
         q, k, v, sc, qc, kc = rope_qkv_hp(*parts, pos, split, theta, stream=stream, norm_w=norm_w, eps=eps)
         o, lse = fwd_bf16_hp(q, k, v, sc, qc, kc, want_lse=want_lse, stream=stream)
     elif path == "bf16":
-        q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype, stream=stream, norm_w=norm_w, eps=eps)
+        q, k, v, _ = rope_qkv(*parts, pos, split, theta, operand_dtype or "fp16", stream=stream, norm_w=norm_w,
+                              eps=eps)
         o, lse = fwd_bf16(q, k, v, want_lse=want_lse, stream=stream)
     elif path == "fp8":
         q, k, v, sc = rope_qkv(*parts, pos, split, theta, "e4m3", stream=stream, norm_w=norm_w, eps=eps)

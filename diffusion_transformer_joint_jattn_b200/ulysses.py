@@ -19,7 +19,8 @@ Ulysses turns a sequence-sharded input into a head-sharded one and back:
 Both exchanges are single ``all_to_all_single`` calls (NCCL over NVLink on
 GPUs) that carry all three streams at once: per destination rank the
 payload is [txt block, img block, ref block].  The attention itself is the
-library's device path (``jattn.joint_attention``); it is a parameter only so
+library's device path (``jattn.joint_attention``, the high-precision pair
+unless ``precise=False`` is passed); it is a parameter only so
 that the exchange logic can be exercised on CPU process groups.
 """
 from __future__ import annotations

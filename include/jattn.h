@@ -324,11 +324,13 @@ jattn_status jattn_fwd_fp8_repair_noalloc(const jattn_shape* shape, const void* 
 
 /*
  * The whole path on HOST buffers, for callers whose inputs and outputs live
- * in host memory: copies in, jattn_rope_qkv + jattn_fwd_bf16 (path JATTN_FP16
- * or JATTN_BF16: the 16-bit operand type) or + jattn_fwd_fp8 (path
- * JATTN_E4M3), copy of O out.  The work is pipelined over the batch: the
- * copies of one batch entry overlap the kernels of another, on two copy
- * streams the library creates once per host thread and device.  The call is
+ * in host memory: copies in, then per chunk the high-precision 16-bit pair
+ * jattn_rope_qkv_hp + jattn_fwd_bf16_hp (path JATTN_FP16), jattn_rope_qkv +
+ * jattn_fwd_bf16 with bf16 operands (path JATTN_BF16) or jattn_rope_qkv +
+ * jattn_fwd_fp8 (path JATTN_E4M3), copy of O out.  The work is pipelined
+ * over (batch entry, head group) chunks: the copies of one chunk overlap the
+ * kernels of another, on two copy streams the library creates once per host
+ * thread and device.  The call is
  * ordered like one operation on `stream`: it starts after the work already
  * enqueued there, and `stream` completes only after O is in host memory.
  *   qkv_*, pos : HOST pointers, layouts as jattn_rope_qkv.  Page-locked

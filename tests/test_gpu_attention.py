@@ -127,31 +127,53 @@ def test_joint_attention_with_qk_norm(cuda_device, case):
 def test_host_buffers_end_to_end(cuda_device, pinned):
     """The public one-call API with host tensors (jattn_joint_attention_host:
     copies in, the path pipelined over the batch, copy out): the same bytes
-    as the device-tensor call, from pageable or pinned host memory."""
+    as the device-tensor call -- the high-precision pair by default, the
+    plain pair on bf16 operands with precise=False -- from pageable or pinned
+    host memory."""
     w = W.BY_NAME["tiny"]
     inp = W.make_inputs(w, 0)
     if pinned:
         inp = {k: (None if v is None else v.pin_memory()) for k, v in inp.items()}
     o_host = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta)
     assert o_host.device.type == "cpu"
-    o_dev, _ = _run_bf16(w, inp, cuda_device, want_lse=False)
-    assert torch.equal(o_host, o_dev.cpu())
+    d = to_device(inp, cuda_device)
+    o_dev = jattn.joint_attention(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta)
+    hp = jattn.rope_qkv_hp(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta)
+    o_hp, _ = jattn.fwd_bf16_hp(*hp)
+    torch.cuda.synchronize()
+    assert torch.equal(o_dev, o_hp)
+    assert torch.equal(o_host, o_hp.cpu())
+    o_plain = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                                    precise=False)
+    o_dev, _ = _run_bf16(w, inp, cuda_device, operand="bf16", want_lse=False)
+    assert torch.equal(o_plain, o_dev.cpu())
+    with pytest.raises(ValueError):
+        jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split, w.theta,
+                              precise=False, operand_dtype="fp16")
 
 
 @pytest.mark.parametrize("path,B,H", [("bf16", 3, 2), ("fp8", 3, 2), ("bf16", 2, 12), ("fp8", 1, 9),
-                                      ("bf16", 2, 5)])
+                                      ("bf16", 2, 5), ("plain", 2, 12), ("bf16", 1, 9)])
 def test_host_entry_pipelined_batch(cuda_device, path, B, H):
     """Every (batch entry, head group) chunk runs as its own (2-D copy in,
     kernels, 2-D copy out) stage on the three streams -- H = 12 splits into
-    6 groups of 2 heads, 9 into 3 groups of 3, 2 and 5 stay whole; the result equals
-    the device entry points' on the whole batch, also when the caller's
-    stream already has work queued and the output buffer is reused."""
+    6 groups of 2 heads, 9 into 3 groups of 3, 2 and 5 stay whole; the result
+    equals the device entry points' on the whole batch (the high-precision
+    pair, whose per-head channel-pair choice and block scales do not depend
+    on the chunking; the plain bf16-operand pair; the e4m3 pair), also when
+    the caller's stream already has work queued and the output buffer is
+    reused."""
     w = W.custom(B=B, H=H, d=128, S_txt=77, grid=9, n_ref=1)
     inp = {k: (None if v is None else v.pin_memory()) for k, v in W.make_inputs(w, 5).items()}
     d = to_device(inp, cuda_device)
+    kw = {}
     if path == "bf16":
-        q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "fp16")
+        hp = jattn.rope_qkv_hp(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta)
+        o_dev, _ = jattn.fwd_bf16_hp(*hp)
+    elif path == "plain":
+        q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "bf16")
         o_dev, _ = jattn.fwd_bf16(q, k, v)
+        path, kw = "bf16", dict(precise=False)
     else:
         q, k, v, sc = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "e4m3")
         o_dev, _ = jattn.fwd_fp8(q, k, v, sc)
@@ -159,7 +181,7 @@ def test_host_entry_pipelined_batch(cuda_device, path, B, H):
     for _ in range(2):
         torch.cuda._sleep(1000000)                 # work already queued on the caller's stream
         o_host = jattn.joint_attention(inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"], inp["pos"], w.split,
-                                       w.theta, path=path, out=out)
+                                       w.theta, path=path, out=out, **kw)
         assert torch.equal(o_host, o_dev.cpu())
     assert jattn.device_status()[0] == jattn.OK
 

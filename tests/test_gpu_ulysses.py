@@ -36,7 +36,7 @@ def test_ulysses_single_rank_nccl(cuda_device):
     dist.init_process_group("nccl", rank=0, world_size=1, device_id=cuda_device)
     try:
         shards = ulysses.shard_streams(streams, 1, 0)
-        out = ulysses.ulysses_attention(shards, d["pos"], w.split, w.theta)
+        out = ulysses.ulysses_attention(shards, d["pos"], w.split, w.theta, precise=False)
         out_hp = ulysses.ulysses_attention(shards, d["pos"], w.split, w.theta, precise=True)
         torch.cuda.synchronize()
     finally:
@@ -46,7 +46,7 @@ def test_ulysses_single_rank_nccl(cuda_device):
     got = gather_rows(torch.cat(out_hp, dim=1), torch.arange(w.S).expand(w.B, w.H, w.S))
     assert rel_l2(got, O) <= BF16_REL_L2
     assert max_abs(got, O) <= BF16_MAX_ABS
-    o = jattn.joint_attention(*streams, d["pos"], w.split, w.theta)
+    o = jattn.joint_attention(*streams, d["pos"], w.split, w.theta, precise=False)
     torch.cuda.synchronize()
     assert torch.equal(torch.cat(out, dim=1), o)
     assert jattn.device_status()[0] == jattn.OK
