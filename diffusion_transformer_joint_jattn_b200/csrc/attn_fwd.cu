@@ -7,7 +7,12 @@
 // path with FP8 query/key and FP8 value.  The page names library kernels only;
 // this kernel is written for B200 from the definition.
 //
-// One CTA computes two 128-row query tiles (t = 0, 1) of one (batch, head):
+// Work items (batch * head, pair of query tiles): a CTA walks items with a
+// stride of the grid size; barrier phases and ring positions run on across
+// items, so the next item's Q load and first Q.K^T overlap the current
+// item's epilogue.  The grid is one CTA per item, or one per SM when items
+// walk only a few key tiles.  Per item the CTA computes two 128-row query
+// tiles (t = 0, 1) of one (batch, head):
 //   warps 0..3  softmax of tile 0, warps 4..7 softmax of tile 1: one thread
 //               per query row (= TMEM lane), online softmax with a lazy
 //               rescale (O and l are rescaled only when the running max grows
@@ -23,9 +28,8 @@
 //   (warps 10, 11 idle: they complete the third warpgroup.)
 // The block starts at 168 registers per thread (384 x 168 = 64512); the
 // MMA/TMA warpgroup then releases registers and the two softmax warpgroups
-// grow (224 / 56 for e4m3 operands, 216 / 72 for the high-precision
-// instance, 208 / 88 for the plain 16-bit one, 200 / 104 when walking a
-// key-tile list; 2 x 128 x softmax + 128 x other = 64512).
+// grow (224 / 56 for e4m3 operands, 216 / 72 for the 16-bit instances at
+// d = 128, 208 / 88 at d = 64; 2 x 128 x softmax + 128 x other = 64512).
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256, 256+d), O_1 [384, 384+d).
 // Because the tensor pipe runs one thread's MMAs in order, the commit that
 // signals S_t(j) also proves PV_t(j-1) finished: O_t is stable for the
@@ -51,17 +55,22 @@ constexpr int kThreads = 384;
 // Register split after setmaxnreg (multiples of 8, together exactly the
 // 384 x 168 the block launches with): ptxas allocates each role's code within
 // its share, and a spill in the single MMA-issuing thread sits on the
-// S -> P -> MMA chain, so each instance gets the split that leaves both its
-// softmax and its MMA / TMA code spill-free (checked with -Xptxas -v).
-template <int KIND, bool HP, bool SPARSE>
+// S -> P -> MMA chain, so each instance gets the split that leaves its
+// softmax and its MMA / TMA code spill-free at d = 128 (checked with
+// -Xptxas -v; the high-precision instance keeps 8 bytes outside the loop).
+template <int D, int KIND, bool HP, bool SPARSE>
 __host__ __device__ constexpr uint32_t regs_softmax() {
-  return KIND == 2 ? 224u : (HP ? 216u : (SPARSE ? 200u : 208u));
+  return KIND == 2 ? 224u : (D == 128 ? 216u : 208u);
 }
-template <int KIND, bool HP, bool SPARSE>
+template <int D, int KIND, bool HP, bool SPARSE>
 __host__ __device__ constexpr uint32_t regs_other() {
-  return (kThreads * 168u - 2u * 128u * regs_softmax<KIND, HP, SPARSE>()) / 128u;
+  return (kThreads * 168u - 2u * 128u * regs_softmax<D, KIND, HP, SPARSE>()) / 128u;
 }
 constexpr uint32_t kTmemCols = 512;
+// Launch one persistent CTA per SM when every item walks at most this many
+// key tiles (the 16-bit pass over a few repaired keys); otherwise one CTA per
+// item, which measured at least as fast for long key walks.
+constexpr int kPersistentMaxKv = 4;
 // Lazy rescale: O and l are rescaled only when a row's running max grows by
 // more than this many log2 units, so P <= 2^threshold in between.  16-bit P
 // has room for 2^15 (fewer rescales); e4m3 P keeps 2^8 so that P * 448 / 2^8
@@ -95,7 +104,7 @@ struct Cfg {
 };
 
 struct __align__(8) Bars {
-  uint64_t q_full;
+  uint64_t q_full, q_empty;
   uint64_t k_full[4], k_empty[4];
   uint64_t v_full[4], v_empty[4];
   uint64_t s_full[NQ], p_full[NQ], o_final[NQ];
@@ -155,6 +164,12 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(d), "f"(c));
   return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
+// The value itself, hidden from the compiler's loop-invariant analysis.
+__device__ __forceinline__ uint32_t opaque(uint32_t x) {
+  uint32_t y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -190,20 +205,25 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int qp = blockIdx.x;                           // pair of query tiles
-  const int bh = blockIdx.y;
-  const int b = bh / p.H, h = bh % p.H;
-  // Key tiles this CTA walks: all n_kv in order, or (block-sparse) the
-  // first kv_count entries of its kv_list row.
-  const int32_t* kv_list = SPARSE ? p.kv_list + (static_cast<size_t>(bh) * gridDim.x + qp) * p.n_kv : nullptr;
-  const int n_kv = SPARSE ? p.kv_count[static_cast<size_t>(bh) * gridDim.x + qp] : p.n_kv;
-  auto kv_tile = [&](int j) {
-    if constexpr (SPARSE) return __ldg(kv_list + j);
+  // Work items: (batch * head, pair of query tiles), pairs fastest; this CTA
+  // takes items blockIdx.x, blockIdx.x + gridDim.x, ...  Every barrier's
+  // phase runs on across items (global step and tile counters).
+  const int n_qp = (p.n_tiles + NQ - 1) / NQ;
+  const int n_items = n_qp * p.B * p.H;
+  // Key tiles of an item: all n_kv in order, or (block-sparse) the first
+  // kv_count entries of its kv_list row.
+  auto item_kv = [&](int it) {
+    if constexpr (SPARSE) return p.kv_count[it];
+    else return p.n_kv;
+  };
+  auto kv_tile = [&](int it, int j) {
+    if constexpr (SPARSE) return __ldg(p.kv_list + static_cast<size_t>(it) * p.n_kv + j);
     else return j;
   };
 
   if (threadIdx.x == 0) {
     mbar_init(&bar->q_full, 1);
+    mbar_init(&bar->q_empty, 1);
     for (int s = 0; s < C::KS; ++s) {
       mbar_init(&bar->k_full[s], 1);
       mbar_init(&bar->k_empty[s], 1);
@@ -234,7 +254,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   const WaitCtl ctl{&bar->abort, p.status, p.timeout_ns};
   if (warp >= 8) {
     // Third warpgroup: producer, MMA issuer and two idle warps.
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(regs_other<KIND, HP, SPARSE>()));
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(regs_other<D, KIND, HP, SPARSE>()));
     if (warp == kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -245,33 +265,41 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         tma_prefetch_desc(&tmQc);
         tma_prefetch_desc(&tmKc);
       }
-      mbar_arrive_expect_tx(&bar->q_full, NQ * (C::TB + C::CT));
-      for (int t = 0; t < NQ; ++t) {
-        for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmQ, &bar->q_full, sQ + t * C::TB + x * C::BOXB, x * C::BOX_ELEMS, (qp * NQ + t) * BM, bh);
-        if constexpr (HP) tma_load_3d(&tmQc, &bar->q_full, sQc + t * C::CT, 0, (qp * NQ + t) * BM, bh);
-      }
-      int nk = 0, nv = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int ks = j % C::KS;
-        if (!mbar_wait(&bar->k_empty[ks], ((j / C::KS) & 1) ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(&bar->k_full[ks], C::TB + C::CT);
-        const int kt = kv_tile(j);
-        for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
-        if constexpr (HP) tma_load_3d(&tmKc, &bar->k_full[ks], sKc + ks * C::CT, 0, kt * BN, bh);
-        nk = j + 1;
-        const int vs = j % C::VS;
-        if (!mbar_wait(&bar->v_empty[vs], ((j / C::VS) & 1) ^ 1, ctl)) break;
-        mbar_arrive_expect_tx(&bar->v_full[vs], C::TB);
-        for (int x = 0; x < C::NBOX; ++x)
-          tma_load_3d(&tmV, &bar->v_full[vs], sV + vs * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
-        nv = j + 1;
+      int nq = 0, nk = 0, nv = 0;                   // loads issued: Q pairs, K tiles, V tiles
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int bh = it / n_qp, qp = it % n_qp;
+        const int n_kv = item_kv(it);
+        // the Q buffer is free once the previous item's Q.K^T are done
+        if (nq > 0 && !mbar_wait(&bar->q_empty, (nq - 1) & 1, ctl)) break;
+        mbar_arrive_expect_tx(&bar->q_full, NQ * (C::TB + C::CT));
+        for (int t = 0; t < NQ; ++t) {
+          for (int x = 0; x < C::NBOX; ++x)
+            tma_load_3d(&tmQ, &bar->q_full, sQ + t * C::TB + x * C::BOXB, x * C::BOX_ELEMS, (qp * NQ + t) * BM, bh);
+          if constexpr (HP) tma_load_3d(&tmQc, &bar->q_full, sQc + t * C::CT, 0, (qp * NQ + t) * BM, bh);
+        }
+        ++nq;
+        for (int j = 0; j < n_kv; ++j) {
+          const int ks = nk % C::KS;
+          if (!mbar_wait(&bar->k_empty[ks], ((nk / C::KS) & 1) ^ 1, ctl)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar->k_full[ks], C::TB + C::CT);
+          const int kt = kv_tile(it, j);
+          for (int x = 0; x < C::NBOX; ++x)
+            tma_load_3d(&tmK, &bar->k_full[ks], sK + ks * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
+          if constexpr (HP) tma_load_3d(&tmKc, &bar->k_full[ks], sKc + ks * C::CT, 0, kt * BN, bh);
+          ++nk;
+          const int vs = nv % C::VS;
+          if (!mbar_wait(&bar->v_empty[vs], ((nv / C::VS) & 1) ^ 1, ctl)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bar->v_full[vs], C::TB);
+          for (int x = 0; x < C::NBOX; ++x)
+            tma_load_3d(&tmV, &bar->v_full[vs], sV + vs * C::TB + x * C::BOXB, x * C::BOX_ELEMS, kt * BN, bh);
+          ++nv;
+        }
       }
       // Drain: every load issued must have landed before the CTA may exit.
-      drain_wait(&bar->q_full, 0, ctl);
-      for (int s = 0; s < C::KS && s < nk; ++s) drain_wait(&bar->k_full[s], ((nk - 1 - s) / C::KS) & 1, ctl);
-      for (int s = 0; s < C::VS && s < nv; ++s) drain_wait(&bar->v_full[s], ((nv - 1 - s) / C::VS) & 1, ctl);
+      if (nq > 0) drain_wait(&bar->q_full, (nq - 1) & 1, ctl);
+      for (int i = nk > C::KS ? nk - C::KS : 0; i < nk; ++i) drain_wait(&bar->k_full[i % C::KS], (i / C::KS) & 1, ctl);
+      for (int i = nv > C::VS ? nv - C::VS : 0; i < nv; ++i) drain_wait(&bar->v_full[i % C::VS], (i / C::VS) & 1, ctl);
     }
     } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------ MMA issuer
@@ -280,9 +308,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       const uint32_t idesc_pv = instr_desc(in_fmt, in_fmt, 1, BM, D);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       bool any_mma = false;
+      // e4m3: the tile bases pass through opaque() so that the descriptors
+      // are formed next to each MMA instead of being hoisted out of the loops
+      // (dozens of 64-bit loop invariants do not fit the 56-register share
+      // of this role; the 16-bit instances measured faster without it).
+      auto base_of = [](uint32_t x) { return FP8 ? opaque(x) : x; };
       auto issue_qk = [&](int t, int ks) {
-        const uint32_t kbase = sKa + ks * C::TB;
-        const uint32_t qbase = sQa + t * C::TB;
+        const uint32_t kbase = base_of(sKa + ks * C::TB);
+        const uint32_t qbase = base_of(sQa + t * C::TB);
 #pragma unroll
         for (int kk = 0; kk < C::QK_STEPS; ++kk) {
           const uint32_t off = (kk * 32) / C::SWB * C::BOXB + (kk * 32) % C::SWB;
@@ -300,7 +333,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         any_mma = true;
       };
       auto issue_pv = [&](int t, int vs, bool acc, int kk0, int kk1) {
-        const uint32_t vbase = sVa + vs * C::TB;
+        const uint32_t vbase = base_of(sVa + vs * C::TB);
 #pragma unroll
         for (int kk = kk0; kk < kk1; ++kk) {
           const uint64_t bdesc = smem_desc(vbase + kk * C::MK * C::SWB, C::BOXB, 8 * C::SWB, C::SWMODE);
@@ -308,33 +341,40 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           else mma_f16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, bdesc, idesc_pv, acc || kk > 0);
         }
       };
-      bool ok = mbar_wait(&bar->q_full, 0, ctl) && mbar_wait(&bar->k_full[0], 0, ctl);
-      if (ok) {
+      int nq = 0, nk = 0, nv = 0, gs = 0;           // items, K tiles, V tiles, softmax steps so far
+      bool ok = true;
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const int n_kv = item_kv(it);
+        ok = mbar_wait(&bar->q_full, nq & 1, ctl) && mbar_wait(&bar->k_full[nk % C::KS], (nk / C::KS) & 1, ctl);
+        if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < NQ; ++t) {
-          issue_qk(t, 0);
+          issue_qk(t, nk % C::KS);
           mma_commit(&bar->s_full[t]);
         }
-        mma_commit(&bar->k_empty[0]);
+        mma_commit(&bar->k_empty[nk % C::KS]);
+        if (n_kv == 1) mma_commit(&bar->q_empty);    // this item's last Q.K^T
+        ++nk;
         for (int j = 0; j < n_kv && ok; ++j) {
-          const int vs = j % C::VS;
-          const int ks = (j + 1) % C::KS;
+          const int vs = nv % C::VS;
+          const int ks = nk % C::KS;
+          const int ph = (gs + j) & 1;                // phase of this step's softmax barriers
           const bool more = j + 1 < n_kv;
-          ok = mbar_wait(&bar->v_full[vs], (j / C::VS) & 1, ctl);
+          ok = mbar_wait(&bar->v_full[vs], (nv / C::VS) & 1, ctl);
           for (int t = 0; t < NQ && ok; ++t) {
             if constexpr (FP8) {
               // P arrives in two halves: the first half's P.V steps overlap
               // the softmax of the second half.
-              ok = mbar_wait(&bar->p_half[t], j & 1, ctl);
+              ok = mbar_wait(&bar->p_half[t], ph, ctl);
               if (!ok) break;
               tc_fence_after();
               issue_pv(t, vs, j > 0, 0, C::PV_STEPS / 2);
-              ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
+              ok = mbar_wait(&bar->p_full[t], ph, ctl);
               if (!ok) break;
               tc_fence_after();
               issue_pv(t, vs, true, C::PV_STEPS / 2, C::PV_STEPS);
             } else {
-              ok = mbar_wait(&bar->p_full[t], j & 1, ctl);
+              ok = mbar_wait(&bar->p_full[t], ph, ctl);
               if (!ok) break;
               tc_fence_after();
               issue_pv(t, vs, j > 0, 0, C::PV_STEPS);
@@ -342,18 +382,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
             if (t == NQ - 1) mma_commit(&bar->v_empty[vs]);
             if (more) {
               if (t == 0) {
-                ok = mbar_wait(&bar->k_full[ks], ((j + 1) / C::KS) & 1, ctl);
+                ok = mbar_wait(&bar->k_full[ks], (nk / C::KS) & 1, ctl);
                 if (!ok) break;
                 tc_fence_after();
               }
               issue_qk(t, ks);
               mma_commit(&bar->s_full[t]);
-              if (t == NQ - 1) mma_commit(&bar->k_empty[ks]);
+              if (t == NQ - 1) {
+                mma_commit(&bar->k_empty[ks]);
+                if (j + 2 == n_kv) mma_commit(&bar->q_empty);   // this item's last Q.K^T
+              }
             } else {
               mma_commit(&bar->o_final[t]);
             }
           }
+          if (!ok) break;
+          ++nv;
+          if (more) ++nk;
         }
+        gs += n_kv;
+        ++nq;
       }
       if (any_mma) {
         mma_commit(&bar->mma_final);
@@ -363,16 +411,26 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     }
   } else {
     // ------------------------------------------------------------ softmax
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(regs_softmax<KIND, HP, SPARSE>()));
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(regs_softmax<D, KIND, HP, SPARSE>()));
     const int t = warp >> 2;                          // query tile of this warpgroup
     const int row = (warp & 3) * 32 + lane;           // TMEM lane == row in the tile
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t ts = tmem + lane_base + col_s(t);
     const uint32_t to = tmem + lane_base + col_o(t);
     const float sl2 = p.scale_log2;
+    // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
+    // exceeds the e4m3 range while p <= 2^8.  HP: as p * (s_v,j / max s_v)
+    // (powers of two; at most 2^15 in fp16).
+    constexpr float kRescaleThreshold = FP8 ? kRescaleThreshold8 : kRescaleThreshold16;
+    const float p8_log2 = FP8 ? 8.8073549220576042f - kRescaleThreshold : 0.f;   // log2(448) - 8
+    bool ok = true;
+    int gs = 0, nq = 0;                                // softmax steps and items so far
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++nq) {
+    const int bh = it / n_qp, qp = it % n_qp;
+    const int b = bh / p.H, h = bh % p.H;
+    const int n_kv = item_kv(it);
     const int q_row = (qp * NQ + t) * BM + row;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
 
     float sq = 1.f, max_sv = 1.f;
     bool unit_scales = false;
@@ -399,15 +457,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // per-tile scale (uniform across the warp).
       if constexpr (HP) unit_scales = __all_sync(0xffffffffu, unit);
     }
-    // FP8: P is stored as p * (s_v,j / max s_v) * 448 / 2^8 so that it never
-    // exceeds the e4m3 range while p <= 2^8.  HP: as p * (s_v,j / max s_v)
-    // (powers of two; at most 2^15 in fp16).
-    constexpr float kRescaleThreshold = FP8 ? kRescaleThreshold8 : kRescaleThreshold16;
-    const float p8_log2 = FP8 ? 8.8073549220576042f - kRescaleThreshold : 0.f;   // log2(448) - 8
     // The K / V block scales of the next tile are fetched one tile ahead so
     // that their load latency stays off the S -> P chain.
     float sk_nxt = 0.f, sv_nxt = 0.f;
-    int kt_cur = n_kv > 0 ? kv_tile(0) : 0;            // key tile of step j
+    int kt_cur = n_kv > 0 ? kv_tile(it, 0) : 0;        // key tile of step j
     if constexpr (SCALED) {
       sk_nxt = sc_k[kt_cur];
       sv_nxt = sc_v[kt_cur];
@@ -415,7 +468,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 
     for (int j = 0; j < n_kv; ++j) {
       const int kt = kt_cur;
-      if (j + 1 < n_kv) kt_cur = kv_tile(j + 1);
+      if (j + 1 < n_kv) kt_cur = kv_tile(it, j + 1);
       float c_j = sl2, bias = 0.f;
       if (SCALED && !unit_scales) {
         c_j = sl2 * sq * sk_nxt;
@@ -428,7 +481,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       // Keys left out of this pass (same for every row of the tile).
       uint4 km = make_uint4(0u, 0u, 0u, 0u);
       if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * p.n_kv + kt);
-      ok = warp_wait(&bar->s_full[t], j & 1, ctl);
+      ok = warp_wait(&bar->s_full[t], (gs + j) & 1, ctl);
       if (!ok) break;
       __syncwarp();
       tc_fence_after();
@@ -553,7 +606,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       mbar_arrive(&bar->p_full[t]);
     }
 
-    if (ok) ok = warp_wait(&bar->o_final[t], 0, ctl);
+    gs += n_kv;
+    if (ok) ok = warp_wait(&bar->o_final[t], nq & 1, ctl);
     if (ok) {
       __syncwarp();
       tc_fence_after();
@@ -609,6 +663,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
       if (p.lse != nullptr && q_row < p.S)
         p.lse[static_cast<size_t>(bh) * p.S + q_row] = lse2 * 0.69314718055994531f;
     }
+    }  // items
   }
 
   tc_fence_before();
@@ -620,6 +675,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
   }
 }
 
+// Streaming multiprocessors of the current device (looked up once per device).
+int sm_count() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 148;
+  if (dev < 64 && cached[dev] > 0) return cached[dev];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
 template <int D, int KIND, bool HP = false, bool SPARSE = false>
 cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                      const CUtensorMap& tqc, const CUtensorMap& tkc, cudaStream_t st) {
@@ -628,7 +695,11 @@ cudaError_t launch_t(const FwdParams& p, const CUtensorMap& tq, const CUtensorMa
   auto kern = attn_fwd_kernel<D, KIND, HP, SPARSE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
   if (e != cudaSuccess) return e;
-  dim3 grid((p.n_tiles + NQ - 1) / NQ, p.B * p.H);
+  // One CTA per work item, or -- when an item walks only a few key tiles and
+  // its set-up and epilogue would dominate -- one persistent CTA per SM.
+  const long long items = static_cast<long long>((p.n_tiles + NQ - 1) / NQ) * p.B * p.H;
+  const bool persistent = p.n_kv <= kPersistentMaxKv && items > sm_count();
+  const int grid = static_cast<int>(persistent ? sm_count() : items);
   kern<<<grid, kThreads, C::SMEM, st>>>(tq, tk, tv, tqc, tkc, p);
   return cudaGetLastError();
 }

@@ -139,8 +139,9 @@ struct FwdParams {
   const uint32_t* kmask;        // null, or [B*H][n_kv][4] words: bit set = key left out of this pass
   const float* lse_prev;        // null, or [B, H, S]: o already holds a partial result with this
                                 // LSE over other keys; the pass merges its own into o (and lse)
-  const int32_t* kv_list;       // null, or [B*H][gridDim.x][n_kv]: the key tiles each CTA (pair of
-  const int32_t* kv_count;      //   query tiles) walks, ascending, and how many ([B*H][gridDim.x])
+  const int32_t* kv_list;       // null, or [B*H][n_qp][n_kv]: the key tiles each pair of query
+  const int32_t* kv_count;      //   tiles walks, ascending, and how many ([B*H][n_qp]); n_qp =
+                                //   ceil(n_tiles / 2); every count >= 1
   uint32_t* status;
   uint64_t timeout_ns;
   long long* trace;             // development timing probe; always null in the library
