@@ -38,14 +38,13 @@ from diffusion_transformer_joint_jattn_b200 import workloads as W  # noqa: E402
 WORKLOAD = "t2i_2048_base"
 # DRAM bytes per launch of the forward kernels on t2i_2048_base: the ncu
 # captures of the same kernels on t2i_1024_base (dram__bytes_read.sum +
-# dram__bytes_write.sum: 205.21 MB with fp16 operands, 109.19 MB with e4m3
-# operands) scaled by the token count 16896 / 4608 (the traffic is Q, K, V
-# and O once each, linear in tokens).
-FWD_TRAFFIC_BYTES = 205.21e6 * 16896 / 4608
-FWD_FP8_TRAFFIC_BYTES = 109.19e6 * 16896 / 4608
-# The high-precision instance (the headline's forward): 184.13 MB read +
-# 35.79 MB written on t2i_1024_base (profiles/attn_fwd_hp_t2i_1024_base.md).
-FWD_HP_TRAFFIC_BYTES = (184.13e6 + 35.79e6) * 16896 / 4608
+# dram__bytes_write.sum: 169.94 + 34.45 MB with fp16 operands, 85.03 + 24.42
+# MB with e4m3 operands, 184.28 + 36.21 MB for the high-precision instance,
+# the headline's forward) scaled by the token count 16896 / 4608 (the
+# traffic is Q, K, V and O once each, linear in tokens).
+FWD_TRAFFIC_BYTES = (169.94e6 + 34.45e6) * 16896 / 4608
+FWD_FP8_TRAFFIC_BYTES = (85.03e6 + 24.42e6) * 16896 / 4608
+FWD_HP_TRAFFIC_BYTES = (184.28e6 + 36.21e6) * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 # Per-sample time of the oracle on the host cores (both CPU legs use the same
@@ -317,7 +316,7 @@ def run_ours(args, rank, world, local):
 
     extras = {}
     if not args.no_extras:
-        extras = measure_extras(jattn, ctx, w, dinp, args, flops, ms8 if fp8 is not None else None)
+        extras = measure_extras(jattn, ctx, w, dinp, args, flops)
         extras["workloads"] = measure_other_workloads(jattn, ctx, args)
 
     e2e = None
@@ -361,15 +360,16 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
-def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops, ms_fp8):
+def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops):
     """The next-row paths on the headline workload, timed the same way
     (device events around the call, inputs resident, workspace allocated
     beforehand):
     * FP8 attention with token repair (the whole call: prologue, selection,
-      gather, masked FP8 pass, merged fp16 pass);
+      gather, masked FP8 pass, merged fp16 pass), in alternation with the
+      plain FP8 step;
     * the prologue with the query/key RMSNorm fused in, against the same
       prologue without it."""
-    out = {"fp8_repair": measure_repair(jattn, ctx, w, dinp, args.rho, args.steps, args.warmup, ms_fp8)}
+    out = {"fp8_repair": measure_repair(jattn, ctx, w, dinp, args.rho, args.steps, args.warmup)}
     out["block_sparse"] = measure_block_sparse(jattn, ctx, w, dinp, args.tau, args.steps, args.warmup)
     B, H, S, d = w.B, w.H, w.S, w.d
     q = torch.empty(B, H, S, d, dtype=torch.float16, device=ctx.dev)
@@ -425,21 +425,44 @@ def measure_block_sparse(jattn, ctx: Ctx, w, dinp, tau, steps, warmup):
             "operands": "fp16 from jattn_rope_qkv (prologue not timed)"}
 
 
-def measure_repair(jattn, ctx: Ctx, w, dinp, rho, steps, warmup, ms_fp8):
+def measure_repair(jattn, ctx: Ctx, w, dinp, rho, steps, warmup):
+    """FP8 with token repair, timed in alternation with the plain FP8 step
+    (one of each per round, each between its own events) so that the
+    overhead compares calls made under the same clock and power state."""
     B, H, S, d = w.B, w.H, w.S, w.d
     n = jattn.repair_count(B, H, w.S_txt, w.S_img, w.S_ref, d, rho)
     ws = torch.empty(jattn.repair_workspace_bytes(B, H, w.S_txt, w.S_img, w.S_ref, d, rho), dtype=torch.uint8,
                      device=ctx.dev)
     o = torch.empty(B, S, H, d, dtype=torch.bfloat16, device=ctx.dev)
-    ms, _ = time_calls(ctx, lambda ev: jattn.fwd_fp8_repair(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"],
-                                                            dinp["pos"], w.split, w.theta, rho=rho, workspace=ws,
-                                                            o=o, stream=ctx.stream), steps, warmup)
+    plain = path_step(jattn, w, dinp, "fp8", ctx.dev, ctx.stream)
+
+    def repair():
+        jattn.fwd_fp8_repair(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                             rho=rho, workspace=ws, o=o, stream=ctx.stream)
+
+    for _ in range(warmup):
+        plain(None)
+        repair()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    ctx.barrier()
+    torch.cuda.synchronize()
+    for e in ev:
+        e[0].record(ctx.stream)
+        plain(None)
+        e[1].record(ctx.stream)
+        e[2].record(ctx.stream)
+        repair()
+        e[3].record(ctx.stream)
+    torch.cuda.synchronize()
+    ctx.barrier()
     code, bits = jattn.device_status(clear=True)
     if code != jattn.OK:
         raise RuntimeError(f"device status {code} bits {bits} after the FP8-with-repair run")
+    ms_p = ctx.max_ranks(float(np.mean([e[0].elapsed_time(e[1]) for e in ev])))
+    ms = ctx.max_ranks(float(np.mean([e[2].elapsed_time(e[3]) for e in ev])))
     return {"value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
             "rho": rho, "repaired_per_head": n, "workspace_bytes": ws.numel(), "gpu_launches_per_step": 5 if n else 2,
-            "overhead_vs_fp8": None if ms_fp8 is None else round(ms / ms_fp8 - 1, 4)}
+            "plain_fp8_ms_interleaved": round(ms_p, 4), "overhead_vs_fp8": round(ms / ms_p - 1, 4)}
 
 
 def measure_other_workloads(jattn, ctx: Ctx, args):
@@ -453,18 +476,15 @@ def measure_other_workloads(jattn, ctx: Ctx, args):
         w = W.BY_NAME[name]
         dinp = {k: (None if v is None else v.to(ctx.dev)) for k, v in W.make_inputs(w, 0).items()}
         res = {"B": w.B, "S": w.S, "flops_per_call": w.flops}
-        ms_fp8 = None
         for path in paths:
             ms, pro, fwd, _, _ = measure_path(jattn, ctx, w, dinp, path, steps, warmup)
-            if path == "fp8":
-                ms_fp8 = ms
             res[path] = {"value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "ms_per_step": round(ms, 4),
                          "prologue_ms": round(pro, 4), "fwd_ms": round(fwd, 4),
                          "roofline": tensor_roofline(w.flops, fwd, peaks, peak_src, path == "fp8", None,
                                                      f"attn_fwd_kernel<128, {'e4m3' if path == 'fp8' else 'fp16'} "
                                                      "operands>")}
         if name == "t2i_2048_distilled":
-            res["fp8_repair"] = measure_repair(jattn, ctx, w, dinp, args.rho, steps, warmup, ms_fp8)
+            res["fp8_repair"] = measure_repair(jattn, ctx, w, dinp, args.rho, steps, warmup)
         out[name] = res
         del dinp
         torch.cuda.empty_cache()
