@@ -57,7 +57,7 @@ constexpr int kThreads = 384;
 // its share, and a spill in the single MMA-issuing thread sits on the
 // S -> P -> MMA chain, so each instance gets the split that leaves its
 // softmax and its MMA / TMA code spill-free at d = 128 (checked with
-// -Xptxas -v; the high-precision instance keeps 8 bytes outside the loop).
+// -Xptxas -v).
 template <int D, int KIND, bool HP, bool SPARSE>
 __host__ __device__ constexpr uint32_t regs_softmax() {
   return KIND == 2 ? 224u : (D == 128 ? 216u : 208u);
@@ -478,9 +478,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           sv_nxt = sc_v[kt_cur];
         }
       }
-      // Keys left out of this pass (same for every row of the tile).
+      // Keys left out of this pass (same for every row of the tile; the e4m3
+      // pass of the repair path has them, the high-precision path never
+      // does).  The next tile's mask is asked into L1 now so that its load
+      // stays off the chain.
       uint4 km = make_uint4(0u, 0u, 0u, 0u);
-      if (p.kmask != nullptr) km = __ldg(reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * p.n_kv + kt);
+      if (!HP && p.kmask != nullptr) {
+        const uint4* kmrow = reinterpret_cast<const uint4*>(p.kmask) + static_cast<size_t>(bh) * p.n_kv;
+        km = __ldg(kmrow + kt);
+        if (j + 1 < n_kv) asm volatile("prefetch.global.L1 [%0];" ::"l"(kmrow + kt_cur));
+      }
       ok = warp_wait(&bar->s_full[t], (gs + j) & 1, ctl);
       if (!ok) break;
       __syncwarp();
