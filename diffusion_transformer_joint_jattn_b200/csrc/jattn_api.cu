@@ -68,7 +68,10 @@ jattn_status check_shape(const jattn_shape* s) {
   if (s->B < 1 || s->H < 1 || s->S_txt < 0 || s->S_img < 0 || s->S_ref < 0) return JATTN_ERR_INVALID_ARG;
   const int64_t S = static_cast<int64_t>(s->S_txt) + s->S_img + s->S_ref;
   if (S < 1 || S > (1 << 24)) return JATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(s->B) * s->H > 65535) return JATTN_ERR_INVALID_ARG;   // grid.y
+  const int64_t BH = static_cast<int64_t>(s->B) * s->H;
+  if (BH > 65535) return JATTN_ERR_INVALID_ARG;                        // grid.y of the per-(b,h) kernels
+  if ((S + 2 * JATTN_BLOCK - 1) / (2 * JATTN_BLOCK) * BH > INT32_MAX)   // forward work items (an int)
+    return JATTN_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return JATTN_ERR_UNSUPPORTED;
   return JATTN_OK;
 }

@@ -65,8 +65,10 @@ typedef enum {
 
 typedef enum { JATTN_BF16 = 0, JATTN_FP16 = 1, JATTN_E4M3 = 2 } jattn_dtype;
 
-/* Problem shape.  S = S_txt + S_img + S_ref >= 1, each part >= 0; B, H >= 1;
- * d in {64, 128}. */
+/* Problem shape.  S = S_txt + S_img + S_ref in [1, 2^24], each part >= 0;
+ * B, H >= 1 with B * H <= 65535 and ceil(S / 256) * B * H < 2^31; d in
+ * {64, 128} (JATTN_ERR_UNSUPPORTED otherwise, JATTN_ERR_INVALID_ARG for the
+ * other limits). */
 typedef struct {
   int32_t B, H, S_txt, S_img, S_ref, d;
 } jattn_shape;

@@ -50,6 +50,8 @@ def shape(B=1, H=1, St=10, Si=0, Sr=0, d=128):
     (dict(d=96), jattn.ERR_UNSUPPORTED),
     (dict(d=256), jattn.ERR_UNSUPPORTED),
     (dict(B=300, H=300), jattn.ERR_INVALID_ARG),         # B*H beyond the grid limit
+    (dict(St=(1 << 24) + 1), jattn.ERR_INVALID_ARG),     # S beyond 2^24
+    (dict(H=65535, St=1 << 24), jattn.ERR_INVALID_ARG),  # 2^16 query-tile pairs x 65535 heads: work items past 2^31
 ])
 def test_fwd_rejects_bad_shapes(args, code):
     lib = jattn.load()
