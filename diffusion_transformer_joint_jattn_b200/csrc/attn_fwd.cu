@@ -24,7 +24,8 @@
 //               tile's softmax overlaps the other tile's tensor work.  With
 //               e4m3 operands P is handed over in two halves of 64 keys, so
 //               the first half's P.V overlaps the second half's softmax.
-//   warp 9      TMA producer: Q tiles once, K_j / V_j into smem rings.
+//   warp 9      TMA producer: the item's Q tiles (once the previous item's
+//               Q.K^T are done), K_j / V_j into smem rings.
 //   (warps 10, 11 idle: they complete the third warpgroup.)
 // The block starts at 168 registers per thread (384 x 168 = 64512); the
 // MMA/TMA warpgroup then releases registers and the two softmax warpgroups
