@@ -131,16 +131,22 @@ __global__ void __launch_bounds__(JATTN_BLOCK) qk_correct_kernel(const CorrParam
   for (int k = 0; k < kCorrPairs; ++k)
     angle_cos_sin(p.pos[3 * t + p.rope.axis[pairs[k]]], p.rope.omega[pairs[k]], cs[k], sn[k]);
   const size_t BHS = static_cast<size_t>(p.BH) * p.S;
+  // All eight channel-pair words (Q and K) are requested before any is used.
+  uint32_t words[2][kCorrPairs];
+#pragma unroll
+  for (int which = 0; which < 2; ++which)
+#pragma unroll
+    for (int k = 0; k < kCorrPairs; ++k)
+      words[which][k] = __ldg(reinterpret_cast<const uint32_t*>(row + (which * p.H + h) * D) + pairs[k]);
 #pragma unroll
   for (int which = 0; which < 2; ++which) {
-    const uint32_t* in = reinterpret_cast<const uint32_t*>(row + (which * p.H + h) * D);
     const float inv2e = 1.0f / p.scales[(static_cast<size_t>(which) * p.BH + bh) * p.nblk + blk];
     float r = 1.f;
     if constexpr (NORM) r = p.norm_r[which * BHS + static_cast<size_t>(bh) * p.S + t];
     __half hi[2 * kCorrPairs], lo[2 * kCorrPairs];
 #pragma unroll
     for (int k = 0; k < kCorrPairs; ++k) {
-      const uint32_t u = __ldg(in + pairs[k]);                       // channels 2p, 2p + 1
+      const uint32_t u = words[which][k];                            // channels 2p, 2p + 1
       float a = bf16_to_f32(static_cast<uint16_t>(u & 0xFFFFu));
       float c = bf16_to_f32(static_cast<uint16_t>(u >> 16));
       if constexpr (NORM) {
