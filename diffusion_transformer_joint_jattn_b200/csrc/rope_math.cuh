@@ -43,9 +43,12 @@ __device__ __forceinline__ void angle_cos_sin(int32_t pos_axis, double omega, fl
 // RMSNorm of one value: x * r * w, with r = 1 / sqrt(mean(x^2) + eps) of its row.
 __device__ __forceinline__ float norm_scale(float x, float r, float w) { return __fmul_rn(__fmul_rn(x, r), w); }
 
-// 1 / sqrt(mean of squares + eps) from a row's fp32 sum of squares.
+// 1 / sqrt(mean of squares + eps) from a row's fp32 sum of squares, by the
+// hardware reciprocal square root (rsqrtf, at most 2 ulp from the exact
+// value; the correctly rounded __frsqrt_rn cost the norm prologue 11%).
+// Every kernel that needs a row's factor reads the one the prologue stored.
 __device__ __forceinline__ float norm_factor(float sum_sq, int d, float eps) {
-  return __frsqrt_rn(__fmaf_rn(sum_sq, 1.0f / static_cast<float>(d), eps));
+  return rsqrtf(__fmaf_rn(sum_sq, 1.0f / static_cast<float>(d), eps));
 }
 
 // (a, b) rotated by the angle with cosine c and sine s.

@@ -13,9 +13,9 @@ oracle, through the C ABI.
 * Standalone quantiser: codes and scales bit-exact (its inputs are exact).
 * Query/key RMSNorm fused in front of the rotation (jattn_rope_qkv_norm): the
   same bounds with the fp32 normalisation's error added (sum of 128 squares
-  and a correctly rounded 1/sqrt: a few 2^-24 relative, bounded here by
-  2^-18 of the pair's magnitude), and a 2^-17 ambiguity window for e4m3
-  codes.
+  and the hardware 1/sqrt, at most 2 ulp: a few 2^-23 relative, bounded
+  here by 2^-18 of the pair's magnitude), and a 2^-17 ambiguity window for
+  e4m3 codes.
 """
 import numpy as np
 import pytest
