@@ -371,6 +371,7 @@ def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops):
       prologue without it."""
     out = {"fp8_repair": measure_repair(jattn, ctx, w, dinp, args.rho, args.steps, args.warmup)}
     out["block_sparse"] = measure_block_sparse(jattn, ctx, w, dinp, args.tau, args.steps, args.warmup)
+    out["torch_sdpa"] = measure_torch_sdpa(jattn, ctx, w, dinp, args.steps, args.warmup)
     B, H, S, d = w.B, w.H, w.S, w.d
     q = torch.empty(B, H, S, d, dtype=torch.float16, device=ctx.dev)
     bufs = (q, torch.empty_like(q), torch.empty_like(q), None)
@@ -423,6 +424,24 @@ def measure_block_sparse(jattn, ctx: Ctx, w, dinp, tau, steps, warmup):
             "dense_equivalent_tflops": round(w.flops / ms / 1e9, 2),
             "kept_tflops": round(kept_flops / ms / 1e9, 2), "gpu_launches_per_call": 3,
             "operands": "fp16 from jattn_rope_qkv (prologue not timed)"}
+
+
+def measure_torch_sdpa(jattn, ctx: Ctx, w, dinp, steps, warmup):
+    """Context only (never an oracle, never the product path): PyTorch's
+    scaled_dot_product_attention, whichever fused backend it picks, on the
+    same rotated fp16 operands laid out [B, H, S, d] by jattn_rope_qkv, beside
+    this library's plain fp16-operand forward on the same operands, timed the
+    same way (device events, inputs resident)."""
+    import torch.nn.functional as F
+    q, k, v, _ = jattn.rope_qkv(dinp["qkv_txt"], dinp["qkv_img"], dinp["qkv_ref"], dinp["pos"], w.split, w.theta,
+                                "fp16")
+    o = torch.empty(w.B, w.S, w.H, w.d, dtype=torch.bfloat16, device=ctx.dev)
+    with torch.cuda.stream(ctx.stream):
+        ms_t, _ = time_calls(ctx, lambda ev: F.scaled_dot_product_attention(q, k, v), steps, warmup)
+    ms_j, _ = time_calls(ctx, lambda ev: jattn.fwd_bf16(q, k, v, o=o, stream=ctx.stream), steps, warmup)
+    return {"ms": round(ms_t, 4), "tflops": round(w.flops / ms_t / 1e9, 2),
+            "jattn_fwd_bf16_ms": round(ms_j, 4), "jattn_fwd_bf16_tflops": round(w.flops / ms_j / 1e9, 2),
+            "torch": torch.__version__, "note": "context only: torch SDPA on the same fp16 [B, H, S, d] operands"}
 
 
 def measure_repair(jattn, ctx: Ctx, w, dinp, rho, steps, warmup):
@@ -583,6 +602,18 @@ def oracle_sample(w, rows_per_head: int, heads: int, seed: int = 0):
     return dt, 4 * heads * rows.shape[-1] * w.S * w.d, workers
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), for the oracle timings."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def host_workers() -> int:
     """Worker threads of the oracle timing: one per host core."""
     return max(1, os.cpu_count() or 1)
@@ -621,7 +652,7 @@ def cpu_baseline(w, target_s: float = ORACLE_SAMPLE_S, samples: int = 2):
         dts.append(dt)
     dt = float(np.mean(dts))
     return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": workers, "blas_threads_per_worker": 1,
-            "kind": "oracle",
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{heads} heads x {rows} sampled query rows of {w.name} (S={w.S}, d={w.d}), FP64 numpy "
                       f"oracle incl. RoPE, mean of {samples} samples of {dt:.1f} s"}
 
@@ -647,7 +678,8 @@ def run_reference(args, rank, world):
                        "note": "each step = FP64 oracle on %d heads x %d sampled rows; ms_per_step extrapolated "
                                "to the full call from the sampled rate" % (heads, rows)},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": workers, "blas_threads_per_worker": 1,
-                             "kind": "oracle", "sample": f"{heads} heads x {rows} query rows per step"},
+                             "kind": "oracle", "cpu_model": cpu_model(),
+                             "sample": f"{heads} heads x {rows} query rows per step"},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
