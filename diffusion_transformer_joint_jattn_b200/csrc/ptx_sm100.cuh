@@ -79,14 +79,21 @@ struct WaitCtl {
 // Wait for the phase with parity `parity` of `bar` to complete.  Returns
 // false (after recording JATTN_DEV_TIMEOUT and raising the CTA's abort flag)
 // if the time limit passes or another role has aborted.
+// The clock is first read after 1024 unsuccessful polls (and then every
+// 1024), not before the first: a %globaltimer read costs hundreds of cycles,
+// which would otherwise sit between a barrier's completion and the waiting
+// thread seeing it.  Each poll suspends for at most a short hardware time
+// slice, so the first reading still comes well inside the limit.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& ctl) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
+  uint64_t t0 = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
+    if ((i & 1023u) == 0) {
       if (*ctl.abort) return false;
-      if (globaltimer_ns() - t0 > ctl.limit_ns) {
+      const uint64_t now = globaltimer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > ctl.limit_ns) {
         atomicOr(ctl.status, JATTN_DEV_TIMEOUT);
         *ctl.abort = 1u;
         return false;
