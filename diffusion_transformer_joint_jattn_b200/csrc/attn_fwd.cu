@@ -507,18 +507,22 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         for (int e = 0; e < BN; ++e)
           if (e >= valid) v[e] = -INFINITY;
       }
+      // Row max as a ternary tree (128 -> 43 -> 15 -> 5 -> 1): five levels of
+      // independent three-input maxima instead of long dependent chains.
       auto row_max = [&]() {
-        float mx0 = v[0], mx1 = v[1], mx2 = v[2], mx3 = v[3];
+        static_assert(BN == 128, "the tree below covers 128 values");
+        float a[43];
 #pragma unroll
-        for (int e = 4; e < BN - 4; e += 8) {
-          mx0 = max3(mx0, v[e + 0], v[e + 1]);
-          mx1 = max3(mx1, v[e + 2], v[e + 3]);
-          mx2 = max3(mx2, v[e + 4], v[e + 5]);
-          mx3 = max3(mx3, v[e + 6], v[e + 7]);
-        }
-        mx0 = max3(mx0, v[BN - 4], v[BN - 3]);
-        mx1 = max3(mx1, v[BN - 2], v[BN - 1]);
-        return fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        for (int i = 0; i < 42; ++i) a[i] = max3(v[3 * i], v[3 * i + 1], v[3 * i + 2]);
+        a[42] = fmaxf(v[126], v[127]);
+        float c[15];
+#pragma unroll
+        for (int i = 0; i < 14; ++i) c[i] = max3(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+        c[14] = a[42];
+        float e[5];
+#pragma unroll
+        for (int i = 0; i < 5; ++i) e[i] = max3(c[3 * i], c[3 * i + 1], c[3 * i + 2]);
+        return max3(e[0], e[1], fmaxf(e[2], fmaxf(e[3], e[4])));
       };
       float mx_raw = row_max();
       // Keys left out of this pass hold zero codes (their logits are exactly
