@@ -548,8 +548,10 @@ def run_partition(args, rank, world, local):
     bsl, g, r = ulysses.rank_work(rank, w.B, cfg, uly)
     inp = W.make_inputs(w, seed=0)
     streams = [None if t is None else t[bsl] for t in (inp["qkv_txt"], inp["qkv_img"], inp["qkv_ref"])]
-    shards = [None if t is None else t.to(dev) for t in ulysses.shard_streams(streams, uly, r)]
-    pos = inp["pos"].to(dev)
+    host_shards = [None if t is None else t.pin_memory() for t in ulysses.shard_streams(streams, uly, r)]
+    shards = [None if t is None else t.to(dev) for t in host_shards]
+    pos_host = inp["pos"].pin_memory()
+    pos = pos_host.to(dev)
 
     def step(ev):
         ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g], precise=True)
@@ -561,6 +563,30 @@ def run_partition(args, rank, world, local):
     code, bits = jattn.device_status(clear=True)
     if code != jattn.OK:
         raise RuntimeError(f"device status {code} bits {bits} on rank {rank}")
+
+    # End to end: every step copies this rank's input shards in from pinned
+    # host memory, runs the same exchange + attention, and copies its output
+    # shards back out (all on the timed stream).
+    outs = ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g], precise=True)
+    out_host = [None if o is None else torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+    def e2e_step(ev):
+        for hs, ds in zip(host_shards, shards):
+            if hs is not None:
+                ds.copy_(hs, non_blocking=True)
+        pos.copy_(pos_host, non_blocking=True)
+        res = ulysses.ulysses_attention(shards, pos, w.split, w.theta, group=groups[g], precise=True)
+        for o, oh in zip(res, out_host):
+            if o is not None:
+                oh.copy_(o, non_blocking=True)
+
+    ms_e2e, _ = time_calls(ctx, e2e_step, args.steps, args.warmup)
+    code, bits = jattn.device_status(clear=True)
+    if code != jattn.OK:
+        raise RuntimeError(f"device status {code} bits {bits} on rank {rank} (end to end)")
+    h2d = world * (sum(t.numel() * t.element_size() for t in host_shards if t is not None)
+                   + pos_host.numel() * pos_host.element_size())
+    d2h = world * sum(t.numel() * t.element_size() for t in out_host if t is not None)
     line = {
         "metric": METRIC, "value": round(whole_job_tflops(w.flops, ms), 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
@@ -572,6 +598,11 @@ def run_partition(args, rank, world, local):
                    "parallelism": f"cfg{cfg} x ulysses{uly}"},
         "gpu_launches": 4 * args.steps,
         "clocks": clocks,
+        "e2e": {"value": round(whole_job_tflops(w.flops, ms_e2e), 2), "unit": UNIT, "ms_per_step": round(ms_e2e, 4),
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "api": "ulysses.ulysses_attention on every rank (high-precision pair), each rank's pinned host "
+                       "input shards copied in and its output shards copied out within the step; bytes summed "
+                       "over ranks"},
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
