@@ -365,7 +365,7 @@ def measure_extras(jattn, ctx: Ctx, w, dinp, args, flops):
     (device events around the call, inputs resident, workspace allocated
     beforehand):
     * FP8 attention with token repair (the whole call: prologue, selection,
-      gather, masked FP8 pass, merged fp16 pass), in alternation with the
+      gather, fp16 pass, masked FP8 pass merging both), in alternation with the
       plain FP8 step;
     * the prologue with the query/key RMSNorm fused in, against the same
       prologue without it."""

@@ -432,6 +432,16 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int n_kv = item_kv(it);
     const int q_row = (qp * NQ + t) * BM + row;
     float m_run = -INFINITY, l_run = 0.f;
+    // Merging into a partial result over other keys (lse_prev given; the
+    // high-precision and block-sparse instances never merge): the row's old
+    // output and its LSE are asked into L2 now, so that the epilogue's reads
+    // of them do not wait on HBM.
+    if (!HP && !SPARSE && p.lse_prev != nullptr && q_row < p.S) {
+      const uint8_t* orow0 = reinterpret_cast<const uint8_t*>(p.o + ((static_cast<size_t>(b) * p.S + q_row) * p.H + h) * D);
+#pragma unroll
+      for (int x = 0; x < D * 2; x += 128) asm volatile("prefetch.global.L2 [%0];" ::"l"(orow0 + x));
+      asm volatile("prefetch.global.L2 [%0];" ::"l"(p.lse_prev + static_cast<size_t>(bh) * p.S + q_row));
+    }
 
     float sq = 1.f, max_sv = 1.f;
     bool unit_scales = false;
@@ -635,7 +645,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           const float mx = fmaxf(la, lse2);
           const float tot = mx + __log2f(ex2_approx(la - mx) + ex2_approx(lse2 - mx));
           w_prev = ex2_approx(la - tot);
-          out_scale *= ex2_approx(lse2 - tot);
+          // a row that saw no key in this pass (l = 0) adds nothing
+          out_scale = l_run > 0.f ? out_scale * ex2_approx(lse2 - tot) : 0.f;
           lse2 = tot;
         }
       }

@@ -579,30 +579,31 @@ jattn_status jattn_fwd_fp8_repair(const jattn_shape* shape, const void* qkv_txt,
     g.status = status_ptr();
     if (jattn::launch_repair_gather(g, cs) != cudaSuccess) return JATTN_ERR_CUDA;
   }
-  // 4. FP8 pass over the other keys.
+  // 4. 16-bit pass over the repaired keys: its partial O and LSE go to o and
+  //    lse_a.  5. FP8 pass over the other keys, merged into them in its
+  //    epilogue through the LSEs (the long pass has time to bring the partial
+  //    rows into L2; the short one would wait on them).
   jattn::FwdParams p{};
   if ((st = fwd_common(shape, ws + L.q8, ws + L.k8, ws + L.v8, o, lse_a, softmax_scale, p)) != JATTN_OK) return st;
-  p.scales = scales;
-  p.kmask = n > 0 ? kmask : nullptr;
   CUtensorMap tq, tk, tv;
   const int kv_rows = jattn::fwd_kv_rows();
+  if (n > 0) {
+    jattn::FwdParams r = p;
+    r.S_kv = n;
+    r.n_kv = n_blocks(n);
+    if ((st = make_map(&tq, ws + L.q16, BH, S, d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
+    if ((st = make_map(&tk, ws + L.kr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
+    if ((st = make_map(&tv, ws + L.vr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
+    if (jattn::launch_fwd_f16(r, d, false, tq, tk, tv, cs) != cudaSuccess) return JATTN_ERR_CUDA;
+  }
+  p.scales = scales;
+  p.kmask = n > 0 ? kmask : nullptr;
+  p.lse_prev = n > 0 ? lse_a : nullptr;
+  p.lse = lse;
   if ((st = make_map(&tq, ws + L.q8, BH, S, d, 1, JATTN_BLOCK)) != JATTN_OK) return st;
   if ((st = make_map(&tk, ws + L.k8, BH, S, d, 1, kv_rows)) != JATTN_OK) return st;
   if ((st = make_map(&tv, ws + L.v8, BH, S, d, 1, kv_rows)) != JATTN_OK) return st;
-  if (jattn::launch_fwd_fp8(p, d, tq, tk, tv, cs) != cudaSuccess) return JATTN_ERR_CUDA;
-  if (n == 0) return JATTN_OK;
-  // 5. 16-bit pass over the repaired keys, merged into o (and lse).
-  jattn::FwdParams r = p;
-  r.scales = nullptr;
-  r.kmask = nullptr;
-  r.S_kv = n;
-  r.n_kv = n_blocks(n);
-  r.lse_prev = lse_a;
-  r.lse = lse;
-  if ((st = make_map(&tq, ws + L.q16, BH, S, d, 2, JATTN_BLOCK)) != JATTN_OK) return st;
-  if ((st = make_map(&tk, ws + L.kr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
-  if ((st = make_map(&tv, ws + L.vr, BH, n, d, 2, kv_rows)) != JATTN_OK) return st;
-  return jattn::launch_fwd_f16(r, d, false, tq, tk, tv, cs) == cudaSuccess ? JATTN_OK : JATTN_ERR_CUDA;
+  return jattn::launch_fwd_fp8(p, d, tq, tk, tv, cs) == cudaSuccess ? JATTN_OK : JATTN_ERR_CUDA;
 }
 
 jattn_status jattn_device_status(void* stream, int clear, uint32_t* bits) {

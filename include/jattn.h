@@ -267,9 +267,9 @@ jattn_status jattn_fwd_block_sparse(const jattn_shape* shape, jattn_dtype in_dty
  * The whole path in one call, on `stream`:
  *   prologue (as jattn_rope_qkv_norm / jattn_rope_qkv with JATTN_E4M3, plus
  *   fp16 Q and the scores) -> selection -> exact fp16 keys / values of the
- *   selected tokens -> FP8 attention over the other keys -> fp16 attention
- *   over the selected keys, merged into o (and lse) through the two partial
- *   log-sum-exps.
+ *   selected tokens -> fp16 attention over the selected keys (a partial o
+ *   and log-sum-exp) -> FP8 attention over the other keys, merged into that
+ *   partial result through the two partial log-sum-exps.
  *   qkv_*, pos, theta, split : as jattn_rope_qkv.
  *   norm_w, eps : query/key RMSNorm as jattn_rope_qkv_norm, or norm_w = NULL.
  *   rho        : 0 <= rho <= 1 (0: plain FP8 path, nothing repaired).
