@@ -651,6 +651,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
         }
       }
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.S + q_row) * p.H + h) * D;
+      // Rows start at multiples of 2 * D bytes from o, so a 32-byte aligned o
+      // makes every 32-byte piece of every row aligned.
+      const bool o_al32 = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r[32];
@@ -661,10 +664,24 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
 #pragma unroll
           for (int e = 0; e < 32; ++e) prev[e] = 0.f;
           if (w_prev != 0.f) {
-            const uint4* src = reinterpret_cast<const uint4*>(orow + c * 32);
+            uint4 pu[4];
+            if (o_al32) {
+#pragma unroll
+              for (int e = 0; e < 2; ++e)
+                asm volatile("ld.global.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                             : "=r"(pu[2 * e].x), "=r"(pu[2 * e].y), "=r"(pu[2 * e].z), "=r"(pu[2 * e].w),
+                               "=r"(pu[2 * e + 1].x), "=r"(pu[2 * e + 1].y), "=r"(pu[2 * e + 1].z),
+                               "=r"(pu[2 * e + 1].w)
+                             : "l"(orow + c * 32 + e * 16)
+                             : "memory");
+            } else {
+              const uint4* src = reinterpret_cast<const uint4*>(orow + c * 32);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) pu[e] = src[e];
+            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const uint4 u = src[e];
+              const uint4 u = pu[e];
               const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
               for (int f = 0; f < 4; ++f) {
@@ -678,9 +695,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
           for (int e = 0; e < 16; ++e)
             w[e] = pack_bf16x2(fmaf(__uint_as_float(r[2 * e]), out_scale, prev[2 * e]),
                                fmaf(__uint_as_float(r[2 * e + 1]), out_scale, prev[2 * e + 1]));
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          if (o_al32) {
+            // 256-bit stores: each writes one whole 32-byte sector of the row
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            for (int e = 0; e < 2; ++e)
+              asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};"
+                           ::"l"(orow + c * 32 + e * 16), "r"(w[8 * e]), "r"(w[8 * e + 1]), "r"(w[8 * e + 2]),
+                             "r"(w[8 * e + 3]), "r"(w[8 * e + 4]), "r"(w[8 * e + 5]), "r"(w[8 * e + 6]),
+                             "r"(w[8 * e + 7])
+                           : "memory");
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
         }
       }
       if (p.lse != nullptr && q_row < p.S)
