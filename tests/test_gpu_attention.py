@@ -254,3 +254,29 @@ def test_long_sequence_and_wide_grid(cuda_device):
     assert rel_l2(got2, O2) <= BF16_REL_L2
     assert max_abs(got2, O2) <= BF16_MAX_ABS
     assert jattn.device_status()[0] == jattn.OK
+
+
+def test_output_only_16_byte_aligned(cuda_device):
+    """The epilogue writes 32-byte pieces of each output row when o is 32-byte
+    aligned and 16-byte pieces otherwise (the C ABI asks only for 16): an o
+    that starts 16 bytes into an allocation gets the same bits, for the plain
+    forward and for the repair path, whose FP8 pass also reads the partial
+    rows back from o."""
+    w = W.custom(B=1, H=3, d=128, S_txt=40, grid=15, n_ref=0)        # S = 265
+    inp = W.make_inputs(w, 5)
+    d = to_device(inp, cuda_device)
+    q, k, v, _ = jattn.rope_qkv(d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta, "fp16")
+    n = w.B * w.S * w.H * w.d
+    flat = torch.empty(n + 8, dtype=torch.bfloat16, device=cuda_device)
+    o16 = flat[8:].view(w.B, w.S, w.H, w.d)                           # 16 bytes past a 256-byte boundary
+    assert o16.data_ptr() % 32 == 16
+    o_ref, _ = jattn.fwd_bf16(q, k, v)
+    jattn.fwd_bf16(q, k, v, o=o16)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, o_ref)
+    args = (d["qkv_txt"], d["qkv_img"], d["qkv_ref"], d["pos"], w.split, w.theta)
+    r_ref = jattn.fwd_fp8_repair(*args, rho=0.05)
+    jattn.fwd_fp8_repair(*args, rho=0.05, o=o16)
+    torch.cuda.synchronize()
+    assert torch.equal(o16, r_ref)
+    assert jattn.device_status()[0] == jattn.OK
