@@ -38,13 +38,13 @@ from diffusion_transformer_joint_jattn_b200 import workloads as W  # noqa: E402
 WORKLOAD = "t2i_2048_base"
 # DRAM bytes per launch of the forward kernels on t2i_2048_base: the ncu
 # captures of the same kernels on t2i_1024_base (dram__bytes_read.sum +
-# dram__bytes_write.sum: 169.94 + 34.45 MB with fp16 operands, 85.03 + 24.42
-# MB with e4m3 operands, 184.28 + 36.21 MB for the high-precision instance,
+# dram__bytes_write.sum: 170.01 + 39.44 MB with fp16 operands, 85.07 + 28.12
+# MB with e4m3 operands, 184.22 + 38.92 MB for the high-precision instance,
 # the headline's forward) scaled by the token count 16896 / 4608 (the
 # traffic is Q, K, V and O once each, linear in tokens).
-FWD_TRAFFIC_BYTES = (169.94e6 + 34.45e6) * 16896 / 4608
-FWD_FP8_TRAFFIC_BYTES = (85.03e6 + 24.42e6) * 16896 / 4608
-FWD_HP_TRAFFIC_BYTES = (184.28e6 + 36.21e6) * 16896 / 4608
+FWD_TRAFFIC_BYTES = (170.01e6 + 39.44e6) * 16896 / 4608
+FWD_FP8_TRAFFIC_BYTES = (85.07e6 + 28.12e6) * 16896 / 4608
+FWD_HP_TRAFFIC_BYTES = (184.22e6 + 38.92e6) * 16896 / 4608
 METRIC = "joint-attention TFLOPS and % of B200 tensor peak (BF16/FP8), 2048^2 shape"
 UNIT = "TFLOPS"
 # Per-sample time of the oracle on the host cores (both CPU legs use the same
