@@ -432,10 +432,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__
     const int n_kv = item_kv(it);
     const int q_row = (qp * NQ + t) * BM + row;
     float m_run = -INFINITY, l_run = 0.f;
-    // Merging into a partial result over other keys (lse_prev given; the
-    // high-precision and block-sparse instances never merge): the row's old
-    // output and its LSE are asked into L2 now, so that the epilogue's reads
-    // of them do not wait on HBM.
+    // Merging into a partial result over other keys (lse_prev given: the
+    // e4m3 pass of the repair path; the high-precision and block-sparse
+    // instances never merge): the row's old output and its LSE are asked
+    // into L2 now, so that the epilogue's reads of them do not wait on HBM.
     if (!HP && !SPARSE && p.lse_prev != nullptr && q_row < p.S) {
       const uint8_t* orow0 = reinterpret_cast<const uint8_t*>(p.o + ((static_cast<size_t>(b) * p.S + q_row) * p.H + h) * D);
 #pragma unroll
