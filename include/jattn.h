@@ -143,7 +143,9 @@ jattn_status jattn_quant_fp8(const jattn_shape* shape, jattn_dtype in_dtype, con
  *   q, k, v : in_dtype (JATTN_FP16 or JATTN_BF16) [B, H, S, d], as written by
  *             jattn_rope_qkv.
  *   o       : bf16 [B, S, H, d] (token-major, ready for the output
- *             projection).
+ *             projection).  16-byte alignment is required; a 32-byte
+ *             aligned o is written with 256-bit stores (fewer store requests,
+ *             same bits).
  *   lse     : fp32 [B, H, S] natural-log sum-exp of the scaled logits, or NULL.
  *   softmax_scale <= 0 selects 1/sqrt(d).
  */
